@@ -1,0 +1,397 @@
+"""Benchmark of the chunked-prefill Block-Union hot path on B200.
+
+One step = one pass of the whole path over one chunk: Block-Union table build
+(``ca_build_block_tables``) + zero-copy paged chunk attention
+(``ca_chunk_attention``) on inputs resident in HBM. The default workload is
+the LLaMA-3.1-8B attention shape (32 query / 8 KV heads, D = 128, 128-token
+blocks) with 128K cached tokens and a 2048-token chunk at 10% per-head mask
+density (synthetic, seeded).
+
+Prints ONE JSON line (rank 0). ``value`` is the effective TFLOP/s of the step
+(4 * D flops per causally visible (row, key) pair inside the selected
+blocks, summed over all ranks' work, divided by the max-over-ranks device
+time). Launch: ``python bench.py --gpus 1 --steps K --warmup W``; for N > 1
+under torchrun (one process per GPU, each runs its own replica of the
+workload: weak scaling, no collective on the data path).
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this path
+has) on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "chunk attn ms & TFLOP/s at 128K ctx (LLaMA-8B shape); speedup vs dense path"
+DEFAULT_WORKLOAD = "llama8b_128k_d10"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def _peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def visible_pairs(tables: np.ndarray, counts: np.ndarray, chunk_start, C: int, blk: int,
+                  G: int, dense_nkv=None) -> int:
+    """(row, key) pairs inside the selected blocks with key <= row position,
+    summed over all query heads (G heads share each group's table)."""
+    B, H_kv = counts.shape
+    total = 0
+    for b in range(B):
+        p = chunk_start[b] + np.arange(C, dtype=np.int64)
+        for g in range(H_kv):
+            if dense_nkv is not None:
+                starts = np.arange(dense_nkv[b], dtype=np.int64) * blk
+            else:
+                starts = tables[b, g, : counts[b, g]].astype(np.int64) * blk
+            if starts.size == 0:
+                continue
+            vis = np.clip(p[:, None] - starts[None, :] + 1, 0, blk)
+            total += int(vis.sum()) * G
+    return total
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ca_clocks_{os.getpid()}_{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    smax.append(float(parts[1]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[4:8]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        finally:
+            try:
+                os.remove(self.path)
+            except OSError:
+                pass
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the fp64 CPU oracle on a bounded sample
+# ---------------------------------------------------------------------------
+
+def oracle_sample_rate(wl, mask, Q, K, V, target_s: float = 15.0, max_rows: int = 4096,
+                       seed: int = 0):
+    """Times the oracle (as it stands) on a seeded sample of query rows sized
+    for about ``target_s`` seconds; returns (TFLOP/s, rows, seconds, threads)."""
+    import oracle
+    T, c, _, _ = oracle.block_tables(mask, wl.group)
+    rng = np.random.default_rng(seed)
+    threads = os.cpu_count() or 1
+    n = 64
+    while True:
+        rows = np.sort(rng.choice(wl.B * wl.H_q * wl.C, size=n, replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attention(Q, K, V, wl.chunk_start, wl.blk, T, c, rows=rows, threads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= target_s * 0.5 or n >= max_rows:
+            break
+        n = min(max_rows, int(n * max(2.0, target_s / max(dt, 1e-3))))
+    # flops of the sampled rows only
+    pairs = 0
+    H_kv = wl.H_kv
+    for flat in rows:
+        r = int(flat % wl.C)
+        h = int((flat // wl.C) % wl.H_q)
+        b = int(flat // (wl.C * wl.H_q))
+        g = h // wl.group
+        p = wl.chunk_start[b] + r
+        starts = T[b, g, : c[b, g]].astype(np.int64) * wl.blk
+        pairs += int(np.clip(p - starts + 1, 0, wl.blk).sum())
+    flops = 4.0 * wl.D * pairs
+    return flops / dt / 1e12, int(rows.size), dt, threads
+
+
+def run_reference(args, wl):
+    import workloads
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    mask = workloads.make_mask(wl)
+    Q, K, V = workloads.make_qkv(wl)
+    vals, rows_used, secs, threads = [], 0, 0.0, 1
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        v, n, dt, threads = oracle_sample_rate(wl, mask, Q, K, V, target_s=per_step, seed=i)
+        if i >= args.warmup:
+            vals.append(v)
+            rows_used += n
+            secs += dt
+    value = statistics.mean(vals)
+    sample = (f"{rows_used} seeded query rows of {wl.B * wl.H_q * wl.C} over {args.steps} steps "
+              f"(fp64 oracle, {secs:.1f} s of CPU time)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs * 1e3 / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(wl),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(wl):
+    return {"workload": wl.name, "B": wl.B, "H_q": wl.H_q, "H_kv": wl.H_kv, "D": wl.D,
+            "block": wl.blk, "chunk": wl.C, "cached_tokens": list(wl.chunk_start),
+            "mask_density": wl.density if wl.density else None,
+            "l2": "256 MB L2 flush between timed steps; K/V cache larger than L2"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    import serving_block_union_b200 as ca
+    import workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    ca.load_library()
+
+    mask_np = workloads.make_mask(wl)
+    Qh, Kh, Vh = workloads.make_qkv(wl)
+    mask = torch.from_numpy(mask_np).to(dev)
+    Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
+    tables = torch.empty((wl.B, wl.H_kv, wl.nKVmax), dtype=torch.int32, device=dev)
+    counts = torch.empty((wl.B, wl.H_kv), dtype=torch.int32, device=dev)
+    O = torch.empty_like(Q)
+    LSE = torch.empty((wl.B, wl.H_q, wl.C), dtype=torch.float32, device=dev)
+    ws = ca.new_workspace(wl.B, wl.H_q, wl.H_kv, wl.C, wl.blk, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def build():
+        ca.build_block_tables(mask, wl.group, tables=tables, counts=counts)
+
+    def attend():
+        ca.chunk_attention(Q, K, V, tables, counts, wl.chunk_start, O=O, LSE=LSE, workspace=ws)
+
+    def dense():
+        ca.dense_chunk_attention(Q, K, V, wl.chunk_start, wl.blk, O=O, LSE=LSE, workspace=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+
+    def timed(fn, n, warm):
+        for _ in range(warm):
+            fn()
+        barrier()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n)]
+        for a, b in ev:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        barrier()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    # work count of one step (from this step's own tables)
+    build()
+    torch.cuda.synchronize(dev)
+    T_np, c_np = tables.cpu().numpy(), counts.cpu().numpy()
+    pairs = visible_pairs(T_np, c_np, wl.chunk_start, wl.C, wl.blk, wl.group)
+    dense_pairs = visible_pairs(T_np, c_np, wl.chunk_start, wl.C, wl.blk, wl.group,
+                                dense_nkv=[-(-(cs + wl.C) // wl.blk) for cs in wl.chunk_start])
+    flops = 4.0 * wl.D * pairs
+    union = float(c_np.sum()) / float(sum(-(-(cs + wl.C) // wl.blk) for cs in wl.chunk_start) * wl.H_kv)
+
+    def step():
+        build()
+        attend()
+
+    gpu_index = local
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        try:
+            gpu_index = int(vis.split(",")[local])
+        except ValueError:
+            gpu_index = local
+    with ClockSampler(gpu_index) as clk:
+        step_ms = timed(step, args.steps, args.warmup)
+        attn_ms = timed(attend, args.steps, args.warmup)
+        build_ms = timed(build, args.steps, args.warmup)
+        dense_ms = timed(dense, args.steps, args.warmup)
+    clocks = clk.summary()
+    assert ca.read_device_status(ws) == ca.CA_OK, "device status not OK"
+
+    # end to end through the public API with pinned host buffers: per step the
+    # chunk's mask, queries and new K/V rows go up, O and LSE come back
+    cs0 = wl.chunk_start
+    mask_h = torch.from_numpy(mask_np).pin_memory()
+    Q_h = Qh.pin_memory()
+    Kc_h = torch.stack([Kh[b, :, cs0[b]:cs0[b] + wl.C] for b in range(wl.B)]).pin_memory()
+    Vc_h = torch.stack([Vh[b, :, cs0[b]:cs0[b] + wl.C] for b in range(wl.B)]).pin_memory()
+    O_h = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    LSE_h = torch.empty(LSE.shape, dtype=LSE.dtype).pin_memory()
+
+    def e2e_step():
+        mask.copy_(mask_h, non_blocking=True)
+        Q.copy_(Q_h, non_blocking=True)
+        for b in range(wl.B):
+            K[b, :, cs0[b]:cs0[b] + wl.C].copy_(Kc_h[b], non_blocking=True)
+            V[b, :, cs0[b]:cs0[b] + wl.C].copy_(Vc_h[b], non_blocking=True)
+        ca.build_block_tables(mask, wl.group, tables=tables, counts=counts)
+        ca.chunk_attention(Q, K, V, tables, counts, wl.chunk_start, O=O, LSE=LSE, workspace=ws)
+        O_h.copy_(O, non_blocking=True)
+        LSE_h.copy_(LSE, non_blocking=True)
+
+    e2e_ms = timed(e2e_step, args.steps, args.warmup)
+    h2d = (mask_h.numel() + Q_h.numel() * 2 + Kc_h.numel() * 2 + Vc_h.numel() * 2)
+    d2h = O_h.numel() * 2 + LSE_h.numel() * 4
+
+    def agg(ms_list):
+        t = torch.tensor([sum(ms_list)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    total_step = agg(step_ms)
+    total_attn = agg(attn_ms)
+    total_build = agg(build_ms)
+    total_dense = agg(dense_ms)
+    total_e2e = agg(e2e_ms)
+    K_ = args.steps
+    value = world * K_ * flops / (total_step * 1e-3) / 1e12
+    attn_tflops = flops / (total_attn / K_ * 1e-3) / 1e12
+    dense_flops = 4.0 * wl.D * dense_pairs
+    peaks, peak_kind = _peaks()
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K_, "warmup": args.warmup, "ms_per_step": total_step / K_,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": _config(wl),
+        "attn_ms": total_attn / K_, "attn_tflops": attn_tflops,
+        "build_us": total_build / K_ * 1e3,
+        "build_gbs": (mask_np.nbytes + 4 * T_np.size + 4 * c_np.size) / (total_build / K_ * 1e-3) / 1e9,
+        "dense_ms": total_dense / K_,
+        "dense_tflops": dense_flops / (total_dense / K_ * 1e-3) / 1e12,
+        "speedup_vs_dense": total_dense / total_step,
+        "union_density": union,
+        "effective_tflop_per_step": flops / 1e12,
+        "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
+                     "unit": "TFLOP/s", "frac": attn_tflops / peak, "traffic": None,
+                     "peak_source": f"{peak_kind} bf16 burst", "kernel": "chunk_attn_kernel"},
+        "e2e": {"value": world * K_ * flops / (total_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": 2 * K_,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n, dt, threads = oracle_sample_rate(wl, mask_np, Qh, Kh, Vh, target_s=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{n} seeded query rows of {wl.B * wl.H_q * wl.C} "
+                                          f"({dt:.1f} s, fp64)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    import workloads
+    wl = workloads.by_name(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

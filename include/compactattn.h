@@ -1,0 +1,144 @@
+/*
+ * compactattn.h — C ABI of the B200 (sm_100a) CompactAttention chunked-prefill
+ * hot path: Block-Union KV table construction and zero-copy paged attention.
+ *
+ * Method: "CompactAttention: Accelerating Chunked Prefill with Block-Union KV
+ * Selection" (arXiv 2605.16839; gist.science / hotpaper.ai / fugumt.com pages,
+ * section "Methodology" / abstract).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All pointers except `chunk_start` are DEVICE pointers owned by the caller.
+ *   The library never allocates, frees or synchronises device memory, except
+ *   ca_read_device_status(), which synchronises its stream.
+ * - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *   default stream) and returns a ca_status. Argument checks run on the host
+ *   before anything is enqueued; on a non-OK return nothing was launched.
+ * - bf16 tensors are raw IEEE bfloat16 (uint16 bit patterns), row-major and
+ *   contiguous in the stated layout; 16-byte aligned base pointers.
+ * - Notation: B sequences, H_q query heads, H_kv KV heads, G = H_q / H_kv
+ *   (query head h reads KV head h / G), D head dim, blk block size (the Q-block
+ *   size, the KV-block size and the cache page size are all blk), C chunk
+ *   length, L_max allocated cache rows per (b, KV head), nKVmax = L_max / blk,
+ *   nQ = C / blk, chunk_start[b] = tokens already cached for sequence b.
+ */
+#ifndef COMPACTATTN_H
+#define COMPACTATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ca_status {
+    CA_OK = 0,
+    CA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, non-finite scale   */
+    CA_ERR_SHAPE = 2,       /* shape precondition violated                          */
+    CA_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned                     */
+    CA_ERR_UNSUPPORTED = 4, /* D, blk or G outside the compiled set                 */
+    CA_ERR_WORKSPACE = 5,   /* workspace NULL, misaligned or smaller than required  */
+    CA_ERR_TABLE = 6,       /* device: table entry/count out of range or unsorted   */
+    CA_ERR_TIMEOUT = 7,     /* device: a bounded wait inside a kernel expired       */
+    CA_ERR_CUDA = 8         /* a CUDA runtime / driver call failed                  */
+} ca_status;
+
+/* Human-readable name of a status code (static storage). */
+const char *ca_status_string(int status);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int ca_version(void);
+
+/*
+ * Block-Union KV table construction (pages: "Methodology", selection stage —
+ * Q-block union, then intra-group union, giving the minimal per-(batch,
+ * KV-group) block table T_{b,g}; the CSR form is the kv_indptr / kv_indices
+ * metadata of the execution stage).
+ *
+ *   U[b,g,j] = OR_{h in group g} OR_{i < nQ} (mask[b,h,i,j] != 0)
+ *   tables[b,g,:]  = the j with U[b,g,j] = 1, ascending, then -1 up to nKVmax
+ *   counts[b,g]    = number of such j
+ *   indptr[k]      = sum of counts over flattened (b,g) < k   (k = 0..B*H_kv)
+ *   indices[...]   = the tables' valid prefixes, concatenated in (b,g) order
+ *
+ * mask    uint8 [B, H_q, nQ, nKVmax], nonzero = tile selected (block j is
+ *         absolute: cached blocks first, then the chunk's).
+ * tables  int32 [B, H_kv, nKVmax]   (H_kv = H_q / group), written in full.
+ * counts  int32 [B, H_kv].
+ * indptr  int32 [B*H_kv + 1] or NULL; indices int32 [B*H_kv*nKVmax] or NULL
+ *         (indices needs indptr). Bit-exact, deterministic.
+ * Errors: CA_ERR_INVALID_ARG (NULL / non-positive), CA_ERR_SHAPE (group does
+ * not divide H_q), CA_ERR_ALIGN (tables/counts/indptr/indices not 4-byte
+ * aligned), CA_ERR_CUDA (launch failure).
+ */
+int ca_build_block_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
+                          int32_t *tables, int32_t *counts, int32_t *indptr, int32_t *indices,
+                          void *stream);
+
+/* Bytes of device workspace ca_chunk_attention / ca_dense_chunk_attention need
+ * for these sizes (a status word plus scheduler state). Allocate it once,
+ * 256-byte aligned and zero-filled; it can be reused by later calls on the
+ * same stream. Returns 0 for invalid sizes. */
+size_t ca_workspace_bytes(int B, int H_q, int H_kv, int C, int blk);
+
+/*
+ * Zero-copy paged chunk attention over the Block-Union tables (pages:
+ * "Methodology", execution stage — dense attention of every query head of the
+ * group over the selected KV blocks, read in place from the KV-head-major
+ * cache [B, H_kv, L, D], with no gather / compaction copy).
+ *
+ * For each sequence b, query head h (g = h / G) and chunk row r, with position
+ * p = chunk_start[b] + r and key set
+ *     K_set = { k : k / blk in T_{b,g}, k <= p }      (causal, bottom-right)
+ * it computes s_k = scale * <Q[b,h,r,:], K[b,g,k,:]> and
+ *     LSE[b,h,r] = ln sum_{k in K_set} exp(s_k)
+ *     O[b,h,r,:] = sum_{k in K_set} exp(s_k - LSE) * V[b,g,k,:]
+ * (O = 0 and LSE = -inf when K_set is empty). Blocks lying wholly after a
+ * row's position are never read. Inputs bf16, products accumulated in fp32,
+ * probabilities rounded to bf16 before the P.V product, O rounded to bf16.
+ *
+ * Q       bf16 [B, H_q, C, D]               (16-byte aligned)
+ * K, V    bf16 [B, H_kv, L_max, D]          (16-byte aligned; rows
+ *         [chunk_start[b], chunk_start[b] + C) already hold the chunk's keys)
+ * tables  int32 [B, H_kv, nKVmax] ascending prefixes (as built above)
+ * counts  int32 [B, H_kv]
+ * chunk_start  HOST int32 [B], 0 <= chunk_start[b], chunk_start[b] + C <= L_max
+ * O       bf16 [B, H_q, C, D] (16-byte aligned), LSE fp32 [B, H_q, C] or NULL
+ * workspace   >= ca_workspace_bytes(...) bytes, 256-byte aligned, zeroed once.
+ * Supported: D in {64, 128}, blk in {64, 128}, G in {1, 2, 4, 8, 16},
+ * 1 <= B <= 128, L_max % blk == 0.
+ * Errors (host): CA_ERR_INVALID_ARG, CA_ERR_SHAPE, CA_ERR_ALIGN,
+ * CA_ERR_UNSUPPORTED, CA_ERR_WORKSPACE, CA_ERR_CUDA. Errors found on the
+ * device (a count outside [0, nKVmax], an entry outside [0, nKVmax) or a
+ * table that is not strictly ascending; an expired bounded wait) never trap:
+ * the kernel records them in the workspace status word, skips or zero-fills
+ * the affected work, and ca_read_device_status() reports them.
+ */
+int ca_chunk_attention(const void *Q, const void *K, const void *V, const int32_t *tables,
+                       const int32_t *counts, const int32_t *chunk_start, int B, int H_q,
+                       int H_kv, int C, int L_max, int D, int blk, float scale, void *O,
+                       float *LSE, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The dense paged path (pages: the "dense attention baseline" the speedup is
+ * quoted against): identical to ca_chunk_attention with
+ * T_{b,g} = [0, ceil((chunk_start[b] + C) / blk)) for every group.
+ * Same arguments minus tables / counts; same errors.
+ */
+int ca_dense_chunk_attention(const void *Q, const void *K, const void *V,
+                             const int32_t *chunk_start, int B, int H_q, int H_kv, int C,
+                             int L_max, int D, int blk, float scale, void *O, float *LSE,
+                             void *workspace, size_t workspace_bytes, void *stream);
+
+/* Synchronises `stream`, then reads the workspace status word written by the
+ * kernels: CA_OK, CA_ERR_TABLE or CA_ERR_TIMEOUT (sticky until the workspace is
+ * zeroed again; CA_ERR_TABLE wins if both are set). CA_ERR_CUDA if the stream
+ * reports an error. Meant for tests and debugging, not the hot path. */
+int ca_read_device_status(const void *workspace, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* COMPACTATTN_H */

@@ -135,7 +135,7 @@ static int attention_row(const attn_job *J, int64_t flat, double *s, int32_t *ke
         if (n_entries < 0 || n_entries > nKVmax) return ORACLE_ETABLE;
         T = J->tables + ((size_t)b * J->H_kv + g) * nKVmax;
     } else {
-        n_entries = (J->chunk_start[b] + C) / blk;  /* nKV_b */
+        n_entries = (J->chunk_start[b] + C + blk - 1) / blk;  /* nKV_b */
     }
 
     int64_t nk = 0;
@@ -218,7 +218,7 @@ int oracle_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *
         return ORACLE_EINVAL;
     if (tables && !counts) return ORACLE_EINVAL;
     for (int b = 0; b < B; ++b)
-        if (chunk_start[b] < 0 || (int64_t)chunk_start[b] + C > L_max || chunk_start[b] % blk)
+        if (chunk_start[b] < 0 || (int64_t)chunk_start[b] + C > L_max)
             return ORACLE_EINVAL;
     if (!rows) n_rows = (int64_t)B * H_q * C;
     for (int64_t i = 0; rows && i < n_rows; ++i)
@@ -267,7 +267,7 @@ int64_t oracle_visible_pairs(const int32_t *tables, const int32_t *counts,
     for (int b = 0; b < B; ++b)
         for (int h = 0; h < H_q; ++h) {
             const int g = h / (H_q / H_kv);
-            const int n = tables ? counts[b * H_kv + g] : (chunk_start[b] + C) / blk;
+            const int n = tables ? counts[b * H_kv + g] : (chunk_start[b] + C + blk - 1) / blk;
             const int32_t *T = tables ? tables + ((size_t)b * H_kv + g) * nKVmax : NULL;
             for (int r = 0; r < C; ++r) {
                 const int64_t p = (int64_t)chunk_start[b] + r;

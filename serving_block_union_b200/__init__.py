@@ -1,0 +1,277 @@
+"""serving_block_union_b200 — B200 (sm_100a) CompactAttention chunked-prefill hot path.
+
+Python binding of ``libcompactattn.so`` (C ABI declared in
+``include/compactattn.h``). This module only marshals arguments: it checks
+dtypes, devices and contiguity, allocates outputs with torch when the caller
+did not pass them, and hands raw pointers plus the current CUDA stream to the
+library. Every step of the path runs in the library's kernels; there is no
+fallback. If the library is missing or fails to load, every call raises.
+
+Entry points (same names as the C ABI, minus the ``ca_`` prefix):
+
+* ``build_block_tables(mask, group)`` — Block-Union tables (selection stage).
+* ``chunk_attention(Q, K, V, tables, counts, chunk_start)`` — zero-copy paged
+  attention over the tables (execution stage).
+* ``dense_chunk_attention(Q, K, V, chunk_start, blk)`` — the dense paged path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+__all__ = [
+    "CAError",
+    "library_path",
+    "load_library",
+    "status_string",
+    "build_block_tables",
+    "workspace_bytes",
+    "new_workspace",
+    "chunk_attention",
+    "dense_chunk_attention",
+    "read_device_status",
+    "EXPORTED_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libcompactattn.so")
+_lock = threading.Lock()
+_lib = None
+
+CA_OK = 0
+CA_ERR_INVALID_ARG = 1
+CA_ERR_SHAPE = 2
+CA_ERR_ALIGN = 3
+CA_ERR_UNSUPPORTED = 4
+CA_ERR_WORKSPACE = 5
+CA_ERR_TABLE = 6
+CA_ERR_TIMEOUT = 7
+CA_ERR_CUDA = 8
+
+EXPORTED_SYMBOLS = (
+    "ca_status_string",
+    "ca_version",
+    "ca_build_block_tables",
+    "ca_workspace_bytes",
+    "ca_chunk_attention",
+    "ca_dense_chunk_attention",
+    "ca_read_device_status",
+)
+
+
+class CAError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_string(status)} ({status})")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load ``libcompactattn.so`` (raises if it is absent: build it with
+    ``python -m serving_block_union_b200.build``)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"{_LIB_PATH} is missing; run `python -m serving_block_union_b200.build`")
+        lib = ctypes.CDLL(_LIB_PATH)
+        P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.ca_status_string.argtypes = [I]
+        lib.ca_status_string.restype = ctypes.c_char_p
+        lib.ca_version.argtypes = []
+        lib.ca_version.restype = I
+        lib.ca_build_block_tables.argtypes = [P, I, I, I, I, I, P, P, P, P, P]
+        lib.ca_build_block_tables.restype = I
+        lib.ca_workspace_bytes.argtypes = [I, I, I, I, I]
+        lib.ca_workspace_bytes.restype = S
+        lib.ca_chunk_attention.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P, P, P, S, P]
+        lib.ca_chunk_attention.restype = I
+        lib.ca_dense_chunk_attention.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, P, P, P, S, P]
+        lib.ca_dense_chunk_attention.restype = I
+        lib.ca_read_device_status.argtypes = [P, P]
+        lib.ca_read_device_status.restype = I
+        _lib = lib
+        return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().ca_status_string(int(status)).decode()
+
+
+# ----------------------------------------------------------------- helpers
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream], device: torch.device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _chunk_start_host(chunk_start, B: int) -> ctypes.Array:
+    if isinstance(chunk_start, torch.Tensor):
+        vals = [int(x) for x in chunk_start.detach().cpu().reshape(-1).tolist()]
+    else:
+        vals = [int(x) for x in chunk_start]
+    if len(vals) != B:
+        raise ValueError(f"chunk_start must have B={B} entries, got {len(vals)}")
+    return (ctypes.c_int32 * B)(*vals)
+
+
+def _check(fn: str, status: int):
+    if status != CA_OK:
+        raise CAError(fn, status)
+
+
+# ----------------------------------------------------------------- tables
+
+def build_block_tables(mask: torch.Tensor, group: int, csr: bool = False,
+                       tables: Optional[torch.Tensor] = None,
+                       counts: Optional[torch.Tensor] = None,
+                       stream: Optional[torch.cuda.Stream] = None):
+    """Block-Union tables of a uint8 / bool mask ``[B, H_q, nQ, nKVmax]``.
+
+    Returns ``(tables int32 [B, H_kv, nKVmax], counts int32 [B, H_kv],
+    indptr int32 [B*H_kv+1] | None, indices int32 [B*H_kv*nKVmax] | None)``;
+    the valid part of ``indices`` is ``indices[:indptr[-1]]``."""
+    if mask.dtype == torch.bool:
+        mask = mask.view(torch.uint8)
+    _need(mask, "mask", torch.uint8, 4)
+    lib = load_library()
+    B, H_q, nQ, nK = mask.shape
+    if group <= 0 or H_q % group:
+        raise ValueError("group must divide H_q")
+    H_kv = H_q // group
+    dev = mask.device
+    if tables is None:
+        tables = torch.empty((B, H_kv, nK), dtype=torch.int32, device=dev)
+    if counts is None:
+        counts = torch.empty((B, H_kv), dtype=torch.int32, device=dev)
+    _need(tables, "tables", torch.int32, 3)
+    _need(counts, "counts", torch.int32, 2)
+    indptr = indices = None
+    if csr:
+        indptr = torch.empty(B * H_kv + 1, dtype=torch.int32, device=dev)
+        indices = torch.empty(B * H_kv * nK, dtype=torch.int32, device=dev)
+    st = lib.ca_build_block_tables(_ptr(mask), B, H_q, nQ, nK, int(group), _ptr(tables),
+                                   _ptr(counts), _ptr(indptr), _ptr(indices),
+                                   _stream_handle(stream, dev))
+    _check("ca_build_block_tables", st)
+    return tables, counts, indptr, indices
+
+
+# ----------------------------------------------------------------- attention
+
+def workspace_bytes(B: int, H_q: int, H_kv: int, C: int, blk: int) -> int:
+    return int(load_library().ca_workspace_bytes(B, H_q, H_kv, C, blk))
+
+
+def new_workspace(B: int, H_q: int, H_kv: int, C: int, blk: int,
+                  device="cuda") -> torch.Tensor:
+    """Zero-filled device workspace for the attention calls (reusable)."""
+    n = workspace_bytes(B, H_q, H_kv, C, blk)
+    if n == 0:
+        raise ValueError("invalid sizes for the workspace")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def _attn_common(Q, K, V, O, LSE, workspace, blk):
+    _need(Q, "Q", torch.bfloat16, 4)
+    _need(K, "K", torch.bfloat16, 4)
+    _need(V, "V", torch.bfloat16, 4)
+    B, H_q, C, D = Q.shape
+    Bk, H_kv, L_max, Dk = K.shape
+    if Bk != B or Dk != D or tuple(V.shape) != tuple(K.shape):
+        raise ValueError(f"shape mismatch: Q {tuple(Q.shape)}, K {tuple(K.shape)}, V {tuple(V.shape)}")
+    dev = Q.device
+    if O is None:
+        O = torch.empty_like(Q)
+    _need(O, "O", torch.bfloat16, 4)
+    if tuple(O.shape) != tuple(Q.shape):
+        raise ValueError("O must have Q's shape")
+    if LSE is None:
+        LSE = torch.empty((B, H_q, C), dtype=torch.float32, device=dev)
+    _need(LSE, "LSE", torch.float32, 3)
+    if workspace is None:
+        workspace = new_workspace(B, H_q, H_kv, C, blk, device=dev)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return B, H_q, H_kv, C, L_max, D, O, LSE, workspace
+
+
+def chunk_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, tables: torch.Tensor,
+                    counts: torch.Tensor, chunk_start: Sequence[int], scale: Optional[float] = None,
+                    O: Optional[torch.Tensor] = None, LSE: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Causal chunk attention over the selected KV blocks, read in place.
+
+    Q bf16 [B, H_q, C, D]; K, V bf16 [B, H_kv, L_max, D]; tables int32
+    [B, H_kv, nKVmax] (blk = L_max / nKVmax); counts int32 [B, H_kv];
+    chunk_start: B host ints. Returns (O bf16 [B, H_q, C, D], LSE fp32 [B, H_q, C])."""
+    _need(tables, "tables", torch.int32, 3)
+    _need(counts, "counts", torch.int32, 2)
+    nK = tables.shape[-1]
+    L_max = K.shape[2]
+    if nK <= 0 or L_max % nK:
+        raise ValueError("tables' last dim must divide L_max (it is L_max / blk)")
+    blk = L_max // nK
+    B, H_q, H_kv, C, L_max, D, O, LSE, workspace = _attn_common(Q, K, V, O, LSE, workspace, blk)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    cs = _chunk_start_host(chunk_start, B)
+    lib = load_library()
+    st = lib.ca_chunk_attention(_ptr(Q), _ptr(K), _ptr(V), _ptr(tables), _ptr(counts), cs, B, H_q,
+                                H_kv, C, L_max, D, blk, float(scale), _ptr(O), _ptr(LSE),
+                                _ptr(workspace), workspace.numel(), _stream_handle(stream, Q.device))
+    _check("ca_chunk_attention", st)
+    return O, LSE
+
+
+def dense_chunk_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                          chunk_start: Sequence[int], blk: int, scale: Optional[float] = None,
+                          O: Optional[torch.Tensor] = None, LSE: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None,
+                          stream: Optional[torch.cuda.Stream] = None
+                          ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """The dense paged path: every block of each sequence's visible length."""
+    B, H_q, H_kv, C, L_max, D, O, LSE, workspace = _attn_common(Q, K, V, O, LSE, workspace, blk)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    cs = _chunk_start_host(chunk_start, B)
+    lib = load_library()
+    st = lib.ca_dense_chunk_attention(_ptr(Q), _ptr(K), _ptr(V), cs, B, H_q, H_kv, C, L_max, D,
+                                      int(blk), float(scale), _ptr(O), _ptr(LSE), _ptr(workspace),
+                                      workspace.numel(), _stream_handle(stream, Q.device))
+    _check("ca_dense_chunk_attention", st)
+    return O, LSE
+
+
+def read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronise and return the sticky device status (CA_OK / CA_ERR_TABLE /
+    CA_ERR_TIMEOUT)."""
+    return int(load_library().ca_read_device_status(_ptr(workspace),
+                                                      _stream_handle(stream, workspace.device)))

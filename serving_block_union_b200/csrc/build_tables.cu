@@ -1,0 +1,197 @@
+// build_tables.cu — Block-Union KV table construction on the GPU.
+//
+// CompactAttention pages, "Methodology", selection stage: the per-head 2D block
+// mask is reduced by a Q-block union (over the chunk's query blocks) and an
+// intra-group union (over the query heads sharing a KV head) into the minimal
+// per-(batch, KV-group) table T_{b,g}; the CSR form is the kv_indptr /
+// kv_indices metadata handed to the paged kernel.
+//
+// One CTA per (b, g). Thread (rg, c) owns 16 consecutive KV blocks (chunk c)
+// and ORs 16-byte vectors of the mask rows rg, rg + RG, ... of the group's
+// G * nQ rows (coalesced: consecutive threads read consecutive 16-byte words
+// of a row). Row groups are OR-combined through shared memory, every chunk
+// turns its 16 bytes into a 16-bit set, and a block-wide exclusive prefix sum
+// of the popcounts (warp shuffles + one shared-memory pass) gives each chunk
+// its write offset, so the table comes out ascending without a sort.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ca_internal.h"
+
+namespace ca {
+
+namespace {
+
+constexpr int kMaxThreads = 1024;
+
+__device__ __forceinline__ uint32_t nonzero_nibble(uint32_t w) {
+    // 4 bits: bit k = (byte k of w != 0)
+    const uint32_t m = __vcmpne4(w, 0u);  // 0xFF in every nonzero byte
+    return ((m >> 7) & 1u) | ((m >> 14) & 2u) | ((m >> 21) & 4u) | ((m >> 28) & 8u);
+}
+
+__device__ __forceinline__ uint32_t nonzero_bytes16(uint4 v) {
+    // bit k of the result = (byte k of v != 0), bytes in memory order
+    return nonzero_nibble(v.x) | (nonzero_nibble(v.y) << 4) | (nonzero_nibble(v.z) << 8) |
+           (nonzero_nibble(v.w) << 12);
+}
+
+// Block-wide exclusive scan of `x` over the first `n_active` threads (a multiple
+// of 32). Returns the exclusive prefix; *total gets the sum.
+__device__ __forceinline__ int block_exclusive_scan(int x, int tid, int n_active, int *warp_sums,
+                                                    int *total) {
+    const int lane = tid & 31, warp = tid >> 5;
+    int incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    const int n_warps = n_active >> 5;
+    if (warp == 0) {
+        int s = lane < n_warps ? warp_sums[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        if (lane < n_warps) warp_sums[lane] = s;  // inclusive over warps
+    }
+    __syncthreads();
+    const int warp_base = warp > 0 ? warp_sums[warp - 1] : 0;
+    *total = warp_sums[n_warps - 1];
+    return warp_base + incl - x;
+}
+
+// chp: chunk threads per row group (multiple of 32), rg: row groups,
+// blockDim.x = chp * rg. vec: mask rows are 16-byte aligned and nKVmax % 16 == 0.
+__global__ void __launch_bounds__(kMaxThreads)
+    union_tables_kernel(const uint8_t *__restrict__ mask, int H_q, int nQ, int nKVmax, int G,
+                        int chp, int rg, int vec, int32_t *__restrict__ tables,
+                        int32_t *__restrict__ counts) {
+    extern __shared__ uint32_t sm_bits[];  // [rg][chp]
+    __shared__ int warp_sums[32];
+    __shared__ int s_base;
+
+    const int bg = blockIdx.x;
+    const int H_kv = H_q / G;
+    const int b = bg / H_kv, g = bg % H_kv;
+    const int tid = threadIdx.x;
+    const int c_local = tid % chp, r_grp = tid / chp;
+    const int n_rows = G * nQ;
+    const int n_chunks = (nKVmax + 15) >> 4;
+    const uint8_t *base = mask + ((size_t)b * H_q + (size_t)g * G) * nQ * (size_t)nKVmax;
+    int32_t *T = tables + (size_t)bg * nKVmax;
+
+    if (tid == 0) s_base = 0;
+    __syncthreads();
+
+    for (int round0 = 0; round0 < n_chunks; round0 += chp) {
+        const int chunk = round0 + c_local;
+        const int j0 = chunk << 4;
+        uint32_t bits = 0;
+        if (chunk < n_chunks) {
+            if (vec) {
+                uint4 acc = make_uint4(0, 0, 0, 0);
+#pragma unroll 8
+                for (int row = r_grp; row < n_rows; row += rg) {
+                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
+                        base + (size_t)row * nKVmax + j0));
+                    acc.x |= v.x; acc.y |= v.y; acc.z |= v.z; acc.w |= v.w;
+                }
+                bits = nonzero_bytes16(acc);
+            } else {
+                const int nb = min(16, nKVmax - j0);
+                for (int row = r_grp; row < n_rows; row += rg) {
+                    const uint8_t *p = base + (size_t)row * nKVmax + j0;
+                    for (int k = 0; k < nb; ++k) bits |= (uint32_t)(__ldg(p + k) != 0) << k;
+                }
+            }
+        }
+        sm_bits[r_grp * chp + c_local] = bits;
+        __syncthreads();
+        int total = 0;
+        if (r_grp == 0) {
+            for (int q = 1; q < rg; ++q) bits |= sm_bits[q * chp + c_local];
+        }
+        // every thread takes part in the scan (barriers inside); only row group 0 counts
+        const int cnt = (r_grp == 0) ? __popc(bits) : 0;
+        const int off = block_exclusive_scan(cnt, tid, chp * rg, warp_sums, &total);
+        if (r_grp == 0 && bits) {
+            int w = s_base + off;
+            uint32_t m = bits;
+            while (m) {
+                const int k = __ffs(m) - 1;
+                T[w++] = j0 + k;
+                m &= m - 1;
+            }
+        }
+        __syncthreads();
+        if (tid == 0) s_base += total;
+        __syncthreads();
+    }
+    const int n = s_base;
+    for (int t = n + tid; t < nKVmax; t += blockDim.x) T[t] = -1;
+    if (tid == 0) counts[bg] = n;
+}
+
+// CSR form: indptr[bg] = sum of counts before bg; indices = valid prefixes.
+__global__ void __launch_bounds__(256)
+    csr_kernel(const int32_t *__restrict__ tables, const int32_t *__restrict__ counts, int n_bg,
+               int nKVmax, int32_t *__restrict__ indptr, int32_t *__restrict__ indices) {
+    __shared__ int red[256];
+    const int bg = blockIdx.x, tid = threadIdx.x;
+    int s = 0;
+    for (int k = tid; k < bg; k += blockDim.x) s += counts[k];
+    red[tid] = s;
+    __syncthreads();
+    for (int w = blockDim.x >> 1; w > 0; w >>= 1) {
+        if (tid < w) red[tid] += red[tid + w];
+        __syncthreads();
+    }
+    const int off = red[0];
+    const int n = counts[bg];
+    if (tid == 0) {
+        indptr[bg] = off;
+        if (bg == n_bg - 1) indptr[n_bg] = off + n;
+    }
+    if (indices) {
+        const int32_t *T = tables + (size_t)bg * nKVmax;
+        for (int t = tid; t < n; t += blockDim.x) indices[off + t] = T[t];
+    }
+}
+
+}  // namespace
+
+int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
+                        int32_t *tables, int32_t *counts, int32_t *indptr, int32_t *indices,
+                        cudaStream_t stream) {
+    const int H_kv = H_q / group;
+    const int n_chunks = (nKVmax + 15) / 16;
+    int chp = ((n_chunks + 31) / 32) * 32;
+    if (chp > kMaxThreads) chp = kMaxThreads;
+    int rg = kMaxThreads / chp;
+    const int n_rows = group * nQ;
+    if (rg > n_rows) rg = n_rows;
+    // keep CTAs modest when the chunk count is small: at most 512 threads
+    while (rg > 1 && chp * rg > 512) --rg;
+    if (rg < 1) rg = 1;
+    const int threads = chp * rg;
+    const int vec = ((reinterpret_cast<uintptr_t>(mask) & 15u) == 0 && (nKVmax % 16) == 0) ? 1 : 0;
+    const size_t smem = sizeof(uint32_t) * (size_t)threads;
+    union_tables_kernel<<<B * H_kv, threads, smem, stream>>>(mask, H_q, nQ, nKVmax, group, chp,
+                                                              rg, vec, tables, counts);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return CA_ERR_CUDA;
+    if (indptr) {
+        csr_kernel<<<B * H_kv, 256, 0, stream>>>(tables, counts, B * H_kv, nKVmax, indptr,
+                                                  indices);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return CA_ERR_CUDA;
+    }
+    return CA_OK;
+}
+
+}  // namespace ca

@@ -1,0 +1,128 @@
+// capi.cu — the extern "C" boundary: host-side argument checks, then one
+// asynchronous launch on the caller's stream. See include/compactattn.h for
+// the contract of every entry point.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "ca_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace {
+
+inline bool aligned(const void *p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+inline bool supported_group(int G) { return G == 1 || G == 2 || G == 4 || G == 8 || G == 16; }
+
+int check_attention(const void *Q, const void *K, const void *V, const int32_t *tables,
+                    const int32_t *counts, bool dense, const int32_t *chunk_start, int B, int H_q,
+                    int H_kv, int C, int L_max, int D, int blk, float scale, const void *O,
+                    const float *LSE, const void *workspace, size_t workspace_bytes) {
+    if (!Q || !K || !V || !O || !chunk_start || !workspace) return CA_ERR_INVALID_ARG;
+    if (!dense && (!tables || !counts)) return CA_ERR_INVALID_ARG;
+    if (B <= 0 || H_q <= 0 || H_kv <= 0 || C <= 0 || L_max <= 0 || D <= 0 || blk <= 0)
+        return CA_ERR_INVALID_ARG;
+    if (!(scale > 0.0f) || !isfinite(scale)) return CA_ERR_INVALID_ARG;
+    if (H_q % H_kv != 0) return CA_ERR_SHAPE;
+    if (L_max % blk != 0) return CA_ERR_SHAPE;
+    for (int b = 0; b < B && b < ca::kMaxBatch; ++b) {
+        const long long cs = chunk_start[b];
+        if (cs < 0 || cs + C > L_max) return CA_ERR_SHAPE;
+    }
+    if (!(D == 64 || D == 128) || !(blk == 64 || blk == 128)) return CA_ERR_UNSUPPORTED;
+    if (!supported_group(H_q / H_kv)) return CA_ERR_UNSUPPORTED;
+    if (B > ca::kMaxBatch) return CA_ERR_UNSUPPORTED;
+    // element counts must stay inside 32-bit TMA coordinates and int indexing
+    if ((long long)B * H_q * C >= (1LL << 31) || (long long)B * H_kv * L_max >= (1LL << 31))
+        return CA_ERR_SHAPE;
+    if (!aligned(Q, 16) || !aligned(K, 16) || !aligned(V, 16) || !aligned(O, 16))
+        return CA_ERR_ALIGN;
+    if ((LSE && !aligned(LSE, 4)) || (tables && !aligned(tables, 4)) ||
+        (counts && !aligned(counts, 4)))
+        return CA_ERR_ALIGN;
+    if (!aligned(workspace, 256) || workspace_bytes < ca_workspace_bytes(B, H_q, H_kv, C, blk))
+        return CA_ERR_WORKSPACE;
+    return CA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ca_status_string(int status) {
+    switch (status) {
+        case CA_OK: return "CA_OK";
+        case CA_ERR_INVALID_ARG: return "CA_ERR_INVALID_ARG";
+        case CA_ERR_SHAPE: return "CA_ERR_SHAPE";
+        case CA_ERR_ALIGN: return "CA_ERR_ALIGN";
+        case CA_ERR_UNSUPPORTED: return "CA_ERR_UNSUPPORTED";
+        case CA_ERR_WORKSPACE: return "CA_ERR_WORKSPACE";
+        case CA_ERR_TABLE: return "CA_ERR_TABLE";
+        case CA_ERR_TIMEOUT: return "CA_ERR_TIMEOUT";
+        case CA_ERR_CUDA: return "CA_ERR_CUDA";
+        default: return "CA_ERR_UNKNOWN";
+    }
+}
+
+int ca_version(void) { return 100; }
+
+size_t ca_workspace_bytes(int B, int H_q, int H_kv, int C, int blk) {
+    if (B <= 0 || H_q <= 0 || H_kv <= 0 || C <= 0 || blk <= 0) return 0;
+    return ca::kWorkspaceHeader;
+}
+
+int ca_build_block_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
+                          int32_t *tables, int32_t *counts, int32_t *indptr, int32_t *indices,
+                          void *stream) {
+    if (!mask || !tables || !counts) return CA_ERR_INVALID_ARG;
+    if (indices && !indptr) return CA_ERR_INVALID_ARG;
+    if (B <= 0 || H_q <= 0 || nQ <= 0 || nKVmax <= 0 || group <= 0) return CA_ERR_INVALID_ARG;
+    if (H_q % group != 0) return CA_ERR_SHAPE;
+    if ((long long)B * H_q * nQ * nKVmax >= (1LL << 40)) return CA_ERR_SHAPE;
+    if ((long long)B * (H_q / group) * nKVmax >= (1LL << 31)) return CA_ERR_SHAPE;
+    if (!aligned(tables, 4) || !aligned(counts, 4) || (indptr && !aligned(indptr, 4)) ||
+        (indices && !aligned(indices, 4)))
+        return CA_ERR_ALIGN;
+    return ca::launch_build_tables(mask, B, H_q, nQ, nKVmax, group, tables, counts, indptr,
+                                   indices, static_cast<cudaStream_t>(stream));
+}
+
+int ca_chunk_attention(const void *Q, const void *K, const void *V, const int32_t *tables,
+                       const int32_t *counts, const int32_t *chunk_start, int B, int H_q,
+                       int H_kv, int C, int L_max, int D, int blk, float scale, void *O,
+                       float *LSE, void *workspace, size_t workspace_bytes, void *stream) {
+    const int st = check_attention(Q, K, V, tables, counts, false, chunk_start, B, H_q, H_kv, C,
+                                   L_max, D, blk, scale, O, LSE, workspace, workspace_bytes);
+    if (st != CA_OK) return st;
+    ca::AttnArgs a{Q, K, V, tables, counts, chunk_start, B, H_q, H_kv, C, L_max, D, blk,
+                   scale, O, LSE, workspace};
+    return ca::launch_chunk_attention(a, false, static_cast<cudaStream_t>(stream));
+}
+
+int ca_dense_chunk_attention(const void *Q, const void *K, const void *V,
+                             const int32_t *chunk_start, int B, int H_q, int H_kv, int C,
+                             int L_max, int D, int blk, float scale, void *O, float *LSE,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    const int st = check_attention(Q, K, V, nullptr, nullptr, true, chunk_start, B, H_q, H_kv, C,
+                                   L_max, D, blk, scale, O, LSE, workspace, workspace_bytes);
+    if (st != CA_OK) return st;
+    ca::AttnArgs a{Q, K, V, nullptr, nullptr, chunk_start, B, H_q, H_kv, C, L_max, D, blk,
+                   scale, O, LSE, workspace};
+    return ca::launch_chunk_attention(a, true, static_cast<cudaStream_t>(stream));
+}
+
+int ca_read_device_status(const void *workspace, void *stream) {
+    if (!workspace) return CA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned int word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof word, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return CA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return CA_ERR_CUDA;
+    if (word & ca::kDevErrTable) return CA_ERR_TABLE;
+    if (word & ca::kDevErrTimeout) return CA_ERR_TIMEOUT;
+    return CA_OK;
+}
+
+}  // extern "C"

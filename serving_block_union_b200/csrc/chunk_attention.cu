@@ -1,0 +1,576 @@
+// chunk_attention.cu — zero-copy paged chunk attention over Block-Union tables
+// (tcgen05 + TMEM + TMA, sm_100a).
+//
+// CompactAttention pages, "Methodology", execution stage: dense attention of
+// every query head of a GQA group over the KV blocks of T_{b,g}, read in place
+// from the KV-head-major cache [B, H_kv, L, D] (each (b, KV head, block) is one
+// contiguous region, so a block is a single TMA box) with no gather copy.
+//
+// Work item (one CTA): (b, g, pair of 128-row tiles). A tile packs G query
+// heads x R = 128 / G chunk rows into the MMA's M = 128 rows (row m = head
+// (m / R), chunk row r0 + (m % R)), so each selected KV block is brought into
+// shared memory once and serves the whole group; the two tiles of the pair
+// share every K/V stage as well. Both tiles' rows lie in the same positions
+// window, so they walk the same prefix of the (ascending) table:
+//   n_eff  = #{t : T[t] <= last position / blk}          (later blocks unread)
+//   n_full = #{t : T[t] <= (first position + 1) / blk - 1} (no causal mask)
+//
+// Warp roles (320 threads, one CTA per SM):
+//   warps 0-3  softmax + epilogue of tile 0 (thread = TMEM lane = packed row)
+//   warps 4-7  softmax + epilogue of tile 1
+//   warp 8     MMA issue (one elected lane) + TMEM allocation
+//   warp 9     TMA producer (Q once, then K and V of T[0..n_eff) in a ring)
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512);
+// P (bf16 pairs) overwrites the first blk/2 columns of S and feeds the P.V MMA
+// straight from tensor memory.
+// MMA order per block j: PV0(j), S0(j+1), PV1(j), S1(j+1): while tile 0's
+// softmax works on S0(j+1) the tensor core runs tile 1's products and the
+// other way round.
+//
+// Online softmax in base 2 (x = s * scale * log2 e); the running max is only
+// raised when it grows by more than 8 (a factor 256), so O is rescaled in
+// TMEM rarely; the final O / l and LSE = (m + log2 l) ln 2 use the same max.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "ca_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace ca {
+
+namespace {
+
+constexpr int kTileM = 128;
+constexpr int kThreads = 320;
+constexpr int kMmaWarp = 8;
+constexpr int kTmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr float kLn2 = 0.693147180559945309f;
+constexpr int kSmemBudget = 227 * 1024;
+constexpr int kSmemFloor = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
+
+struct Params {
+    int B, H_q, H_kv, C, L_max, G, R, n_pairs, nKVmax;
+    float scale_log2;
+    const int32_t *tables;
+    const int32_t *counts;
+    uint16_t *O;
+    float *LSE;
+    unsigned int *status;
+    int chunk_start[kMaxBatch];
+    unsigned char b_order[kMaxBatch];
+};
+
+template <int D, int BLK>
+struct Layout {
+    static constexpr int kQTile = kTileM * D * 2;  // D/64 sub-tiles of 128 rows x 128 B
+    static constexpr int kKV = BLK * D * 2;        // D/64 sub-tiles of BLK rows x 128 B
+    static constexpr int kStagesFit = (kSmemBudget - 2048 - 2 * kQTile) / (2 * kKV);
+    static constexpr int kStages = kStagesFit > 4 ? 4 : kStagesFit;
+    static constexpr int kQOff = 0;
+    static constexpr int kKOff = 2 * kQTile;
+    static constexpr int kVOff = kKOff + kStages * kKV;
+    static constexpr int kBarOff = kVOff + kStages * kKV;
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1;
+    static constexpr int kEnd = kBarOff + kNumBars * 8 + 16;
+    static constexpr int kDynamic = (kEnd + 1024) > kSmemFloor ? (kEnd + 1024) : kSmemFloor;
+    static_assert(kStages >= 2, "need at least two K/V stages");
+    static_assert(kDynamic <= kSmemBudget, "shared memory budget exceeded");
+};
+
+// Entries of the ascending prefix T[0, n) that are <= bound; warp-cooperative
+// (all 32 lanes), scanning windows of 32 from the end (the answer is normally
+// in the last window: only blocks inside the chunk can lie past the bound).
+__device__ __forceinline__ int count_le(const int32_t *T, int n, int bound, int lane) {
+    int hi = n;
+    while (hi > 0) {
+        const int lo = hi > 32 ? hi - 32 : 0;
+        const int idx = lo + lane;
+        const int v = idx < hi ? __ldg(T + idx) : 0;
+        const unsigned gt = __ballot_sync(0xffffffffu, idx < hi && v > bound);
+        const int ngt = __popc(gt);
+        if (ngt < hi - lo) return hi - ngt;
+        hi = lo;
+    }
+    return 0;
+}
+
+template <int D, int BLK, bool DENSE>
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params P) {
+    using L = Layout<D, BLK>;
+    constexpr int NST = L::kStages;
+    constexpr int DCH = D / 64;  // 64-element (128-byte) sub-tiles along D
+    constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, BLK, false);
+    constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, true);
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(smem);
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
+    uint64_t *q_full = bars;
+    uint64_t *k_full = bars + 1;
+    uint64_t *k_empty = k_full + NST;
+    uint64_t *v_full = k_empty + NST;
+    uint64_t *v_empty = v_full + NST;
+    uint64_t *s_full = v_empty + NST;  // [2]
+    uint64_t *p_full = s_full + 2;     // [2]
+    uint64_t *o_full = p_full + 2;     // [2]
+    uint64_t *mma_done = o_full + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---- work item
+    const int per_b = P.H_kv * P.n_pairs;
+    const int b = P.b_order[blockIdx.x / per_b];
+    const int rem = blockIdx.x % per_b;
+    const int pair = rem / P.H_kv;
+    const int g = rem % P.H_kv;
+    const int cs = P.chunk_start[b];
+    const int R = P.R;
+    const int r0 = pair * 2 * R;
+    const int r_end = min(r0 + 2 * R, P.C);
+    const int p_min = cs + r0;
+    const int p_max = cs + r_end - 1;
+    const int jlast = p_max / BLK;
+    const int jfull = (p_min + 1) / BLK - 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(k_full + s, 1);
+            mbar_init(k_empty + s, 1);
+            mbar_init(v_full + s, 1);
+            mbar_init(v_empty + s, 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(s_full + t, 1);
+            mbar_init(p_full + t, 4);
+            mbar_init(o_full + t, 1);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kTmaWarp && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const AbortState ab{abort_flag, P.status};
+
+    // ---- table prefix this item walks (every role computes it the same way)
+    const int32_t *T = nullptr;
+    int n_eff, n_full;
+    if (DENSE) {
+        n_eff = jlast + 1;
+        n_full = jfull + 1 > 0 ? jfull + 1 : 0;
+    } else {
+        int cnt = __ldg(P.counts + b * P.H_kv + g);
+        if (cnt < 0 || cnt > P.nKVmax) {
+            if (threadIdx.x == 0) atomicOr(P.status, kDevErrTable);
+            cnt = 0;
+        }
+        T = P.tables + ((size_t)b * P.H_kv + g) * P.nKVmax;
+        n_eff = count_le(T, cnt, jlast, lane);
+        n_full = count_le(T, n_eff, jfull, lane);
+    }
+
+    if (warp == kTmaWarp) {
+        // ================================================================ producer
+        int k_issued = 0, v_issued = 0;  // loads started (for the drain below)
+        bool q_issued = false;
+        if (n_eff > 0) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(q_full, 2 * L::kQTile);
+                for (int t = 0; t < 2; ++t)
+                    for (int dc = 0; dc < DCH; ++dc)
+                        tma_load_3d(smem + L::kQOff + t * L::kQTile + dc * (kTileM * 128), &tmQ,
+                                    q_full, dc * 64, r0 + t * R, b * P.H_q + g * P.G);
+            }
+            q_issued = true;
+            int prev_last = -1;
+            bool ok = true;
+            for (int w0 = 0; w0 < n_eff && ok; w0 += 32) {
+                const int jj = w0 + lane;
+                const int nwin = min(32, n_eff - w0);
+                int jb = DENSE ? jj : (lane < nwin ? __ldg(T + jj) : 0);
+                if (!DENSE) {
+                    int prv = __shfl_up_sync(0xffffffffu, jb, 1);
+                    if (lane == 0) prv = prev_last;
+                    const bool out = jb < 0 || jb >= P.nKVmax;
+                    const bool bad = lane < nwin && (out || jb <= prv);
+                    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(P.status, kDevErrTable);
+                    prev_last = __shfl_sync(0xffffffffu, jb, nwin - 1);
+                    // an out-of-range entry is fetched from one block past the cache end:
+                    // the copy lands zero-filled and nothing outside K / V is touched
+                    if (out) jb = P.nKVmax;
+                }
+                for (int q = 0; q < nwin; ++q) {
+                    const int blk_idx = __shfl_sync(0xffffffffu, jb, q);
+                    const int j = w0 + q;
+                    const int s = j % NST;
+                    const uint32_t ph = ((j / NST) & 1) ^ 1;
+                    int good = 1;
+                    if (lane == 0) {
+                        good = mbar_wait(k_empty + s, ph, ab);
+                        if (good) {
+                            mbar_arrive_expect_tx(k_full + s, L::kKV);
+                            for (int dc = 0; dc < DCH; ++dc)
+                                tma_load_3d(smem + L::kKOff + s * L::kKV + dc * (BLK * 128), &tmK,
+                                            k_full + s, dc * 64, blk_idx * BLK, b * P.H_kv + g);
+                            k_issued = j + 1;
+                            good = mbar_wait(v_empty + s, ph, ab);
+                        }
+                        if (good) {
+                            mbar_arrive_expect_tx(v_full + s, L::kKV);
+                            for (int dc = 0; dc < DCH; ++dc)
+                                tma_load_3d(smem + L::kVOff + s * L::kKV + dc * (BLK * 128), &tmV,
+                                            v_full + s, dc * 64, blk_idx * BLK, b * P.H_kv + g);
+                            v_issued = j + 1;
+                        }
+                    }
+                    good = __shfl_sync(0xffffffffu, good, 0);
+                    if (!good) {
+                        ok = false;
+                        break;
+                    }
+                }
+            }
+        }
+        // drain: every copy this warp started has landed before the CTA exits
+        if (lane == 0) {
+            if (q_issued) mbar_wait_drain(q_full, 0);
+            for (int j = k_issued > NST ? k_issued - NST : 0; j < k_issued; ++j)
+                mbar_wait_drain(k_full + j % NST, (j / NST) & 1);
+            for (int j = v_issued > NST ? v_issued - NST : 0; j < v_issued; ++j)
+                mbar_wait_drain(v_full + j % NST, (j / NST) & 1);
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ================================================================ MMA issue
+        if (n_eff > 0 && lane == 0) {
+            const uint32_t q_addr = sbase + L::kQOff;
+            const uint32_t k_addr = sbase + L::kKOff;
+            const uint32_t v_addr = sbase + L::kVOff;
+            auto issue_s = [&](int t, int slot) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 B inside the swizzle row
+                    const uint64_t a = sdesc_sw128(
+                        q_addr + t * L::kQTile + (kk >> 2) * (kTileM * 128) + off, 16, 1024);
+                    const uint64_t bb = sdesc_sw128(
+                        k_addr + slot * L::kKV + (kk >> 2) * (BLK * 128) + off, 16, 1024);
+                    mma_ss(tmem + t * 128, a, bb, kIdescS, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_pv = [&](int t, int slot, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < BLK / 16; ++kk) {
+                    const uint64_t bb =
+                        sdesc_sw128(v_addr + slot * L::kKV + kk * (16 * 128), BLK * 128, 1024);
+                    mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bb, kIdescPV,
+                           (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            bool ok = mbar_wait(q_full, 0, ab) && mbar_wait(k_full, 0, ab);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                tc_commit(s_full + 0);
+                issue_s(1, 0);
+                tc_commit(s_full + 1);
+                tc_commit(k_empty + 0);
+            }
+            for (int j = 0; j < n_eff && ok; ++j) {
+                const int s = j % NST;
+                const uint32_t ph = (j / NST) & 1;
+                const bool more = j + 1 < n_eff;
+                const int s1 = (j + 1) % NST;
+                const uint32_t ph1 = ((j + 1) / NST) & 1;
+                if (!(ok = mbar_wait(v_full + s, ph, ab))) break;
+                if (!(ok = mbar_wait(p_full + 0, j & 1, ab))) break;
+                tc_fence_after();
+                issue_pv(0, s, j > 0);
+                if (more) {
+                    if (!(ok = mbar_wait(k_full + s1, ph1, ab))) break;
+                    tc_fence_after();
+                    issue_s(0, s1);
+                    tc_commit(s_full + 0);
+                } else {
+                    tc_commit(o_full + 0);
+                }
+                if (!(ok = mbar_wait(p_full + 1, j & 1, ab))) break;
+                tc_fence_after();
+                issue_pv(1, s, j > 0);
+                tc_commit(v_empty + s);
+                if (more) {
+                    issue_s(1, s1);
+                    tc_commit(s_full + 1);
+                    tc_commit(k_empty + s1);
+                } else {
+                    tc_commit(o_full + 1);
+                }
+            }
+            // drain: all MMAs issued by this thread have completed
+            tc_commit(mma_done);
+            mbar_wait_drain(mma_done, 0);
+        }
+        __syncwarp();
+    } else {
+        // ================================================================ softmax
+        const int t = warp >> 2;
+        const int qw = warp & 3;
+        const int m = qw * 32 + lane;
+        const int h_local = m / R;
+        const int r = r0 + t * R + (m % R);
+        const bool valid = r < P.C;
+        const int p = cs + r;
+        const int h = g * P.G + h_local;
+        const uint32_t lane_base = static_cast<uint32_t>(qw * 32) << 16;
+        const uint32_t tS = tmem + lane_base + t * 128;
+        const uint32_t tO = tmem + lane_base + 256 + t * 128;
+        const float sl2 = P.scale_log2;
+
+        float m_run = -INFINITY, l_run = 0.0f;
+        bool ok = true;
+        for (int j = 0; j < n_eff; ++j) {
+            ok = mbar_wait(s_full + t, j & 1, ab);
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            float s[BLK];
+#pragma unroll
+            for (int c = 0; c < BLK / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tS + c * 32, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(v[i]);
+            }
+            if (j >= n_full) {
+                int jb = DENSE ? j : __ldg(T + j);
+                jb = min(max(jb, 0), P.nKVmax);  // only matters for a flagged, invalid table
+                const int lim = p - jb * BLK;    // keys jb*BLK + c with c <= lim are visible
+#pragma unroll
+                for (int c = 0; c < BLK; ++c)
+                    if (c > lim) s[c] = -INFINITY;
+            }
+            float mx = s[0];
+#pragma unroll
+            for (int c = 1; c < BLK; ++c) mx = fmaxf(mx, s[c]);
+            const float m_blk = mx * sl2;
+            const float m_new = fmaxf(m_run, m_blk);
+            const bool old_finite = m_run != -INFINITY;
+            const bool upd = old_finite ? (m_new > m_run + kRescaleThreshold)
+                                        : (m_new != -INFINITY);
+            float alpha = 1.0f;
+            if (upd) {
+                alpha = old_finite ? ex2_approx(m_run - m_new) : 0.0f;
+                m_run = m_new;
+            }
+            const float m_use = m_run == -INFINITY ? 0.0f : m_run;
+            l_run *= alpha;
+            float sum = 0.0f;
+#pragma unroll
+            for (int c = 0; c < BLK / 64; ++c) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * i], sl2, -m_use));
+                    const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -m_use));
+                    sum += p0 + p1;
+                    pk[i] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(tS + c * 32, pk);
+            }
+            l_run += sum;
+            // O rescale (rare: only when a row's max grew past the threshold). O is
+            // stable here: S(j) was committed after P.V(j-1) was issued.
+            const bool need = upd && old_finite && j > 0;
+            if (__any_sync(0xffffffffu, need)) {
+                const float a = need ? alpha : 1.0f;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld32(tO + c * 32, v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
+                    tmem_st32(tO + c * 32, v);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(p_full + t);
+        }
+        bool have_o = false;
+        if (n_eff > 0 && __all_sync(0xffffffffu, ok)) {
+            const bool got = mbar_wait(o_full + t, 0, ab);
+            have_o = __all_sync(0xffffffffu, got);
+            tc_fence_after();
+        }
+        const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+        uint16_t *orow = P.O + (((size_t)b * P.H_q + h) * P.C + r) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+            uint32_t v[32];
+            if (have_o) {
+                tmem_ld32(tO + c * 32, v);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0u;
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l,
+                                    __uint_as_float(v[2 * i + 1]) * inv_l);
+            if (valid) {
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+        }
+        if (valid && P.LSE != nullptr) {
+            P.LSE[((size_t)b * P.H_q + h) * P.C + r] =
+                (l_run > 0.0f && have_o) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool encode_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
+               uint32_t b0, uint32_t b1, uint32_t b2) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, int BLK, bool DENSE>
+int launch_t(const AttnArgs &a, cudaStream_t stream) {
+    using L = Layout<D, BLK>;
+    auto kern = chunk_attn_kernel<D, BLK, DENSE>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        L::kDynamic);
+    });
+    if (attr_err != cudaSuccess) return CA_ERR_CUDA;
+
+    const int G = a.H_q / a.H_kv;
+    const int R = kTileM / G;
+    const int n_tiles = (a.C + R - 1) / R;
+    const int n_pairs = (n_tiles + 1) / 2;
+
+    CUtensorMap tq, tk, tv;
+    if (!encode_3d(&tq, a.Q, (uint64_t)D, (uint64_t)a.C, (uint64_t)a.B * a.H_q, 64, R, G) ||
+        !encode_3d(&tk, a.K, (uint64_t)D, (uint64_t)a.L_max, (uint64_t)a.B * a.H_kv, 64, BLK, 1) ||
+        !encode_3d(&tv, a.V, (uint64_t)D, (uint64_t)a.L_max, (uint64_t)a.B * a.H_kv, 64, BLK, 1))
+        return CA_ERR_CUDA;
+
+    Params P;
+    P.B = a.B;
+    P.H_q = a.H_q;
+    P.H_kv = a.H_kv;
+    P.C = a.C;
+    P.L_max = a.L_max;
+    P.G = G;
+    P.R = R;
+    P.n_pairs = n_pairs;
+    P.nKVmax = a.L_max / BLK;
+    P.scale_log2 = a.scale * 1.4426950408889634f;
+    P.tables = a.tables;
+    P.counts = a.counts;
+    P.O = static_cast<uint16_t *>(a.O);
+    P.LSE = a.LSE;
+    P.status = static_cast<unsigned int *>(a.workspace);
+    // longest sequences first: their items are the heaviest
+    int order[kMaxBatch];
+    for (int i = 0; i < a.B; ++i) order[i] = i;
+    for (int i = 1; i < a.B; ++i) {
+        const int x = order[i];
+        int k = i - 1;
+        while (k >= 0 && a.chunk_start[order[k]] < a.chunk_start[x]) {
+            order[k + 1] = order[k];
+            --k;
+        }
+        order[k + 1] = x;
+    }
+    for (int i = 0; i < kMaxBatch; ++i) {
+        P.chunk_start[i] = i < a.B ? a.chunk_start[i] : 0;
+        P.b_order[i] = static_cast<unsigned char>(i < a.B ? order[i] : 0);
+    }
+    const unsigned grid = static_cast<unsigned>(a.B * a.H_kv * n_pairs);
+    kern<<<grid, kThreads, L::kDynamic, stream>>>(tq, tk, tv, P);
+    return cudaGetLastError() == cudaSuccess ? CA_OK : CA_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_chunk_attention(const AttnArgs &a, bool dense, cudaStream_t stream) {
+#define CA_DISPATCH(D_, BLK_)                                                    \
+    if (a.D == D_ && a.blk == BLK_)                                              \
+        return dense ? launch_t<D_, BLK_, true>(a, stream) : launch_t<D_, BLK_, false>(a, stream);
+    CA_DISPATCH(128, 128)
+    CA_DISPATCH(128, 64)
+    CA_DISPATCH(64, 128)
+    CA_DISPATCH(64, 64)
+#undef CA_DISPATCH
+    return CA_ERR_UNSUPPORTED;
+}
+
+}  // namespace ca

@@ -1,0 +1,121 @@
+"""The C-ABI library: it loads, exports every symbol ``include/*.h`` declares,
+and rejects bad arguments on the host with the documented status codes.
+No compute call is made here (every case below fails its host-side checks
+before anything is enqueued)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import serving_block_union_b200 as ca
+from serving_block_union_b200 import build as ca_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    ca_build.build()
+    return ca.load_library()
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(ca_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_functions()
+    assert {"ca_build_block_tables", "ca_chunk_attention", "ca_dense_chunk_attention"} <= declared
+    for name in sorted(declared):
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert set(ca.EXPORTED_SYMBOLS) <= declared
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "CA_OK"), (1, "CA_ERR_INVALID_ARG"), (2, "CA_ERR_SHAPE"),
+                       (3, "CA_ERR_ALIGN"), (4, "CA_ERR_UNSUPPORTED"), (5, "CA_ERR_WORKSPACE"),
+                       (6, "CA_ERR_TABLE"), (7, "CA_ERR_TIMEOUT"), (8, "CA_ERR_CUDA")]:
+        assert ca.status_string(code) == name
+    assert ca.status_string(99) == "CA_ERR_UNKNOWN"
+    assert lib.ca_version() >= 100
+
+
+def test_workspace_bytes(lib):
+    n = lib.ca_workspace_bytes(1, 32, 8, 2048, 128)
+    assert n >= 16 and n % 256 == 0
+    assert lib.ca_workspace_bytes(0, 32, 8, 2048, 128) == 0
+
+
+# Fake device addresses: never dereferenced because every call below fails
+# its host-side checks first.
+A16 = ctypes.c_void_p(1 << 20)
+A_MIS = ctypes.c_void_p((1 << 20) + 2)
+
+
+def _attn(lib, **kw):
+    a = dict(Q=A16, K=A16, V=A16, tables=A16, counts=A16, B=1, H_q=32, H_kv=8, C=2048,
+             L_max=34816, D=128, blk=128, scale=0.088, O=A16, LSE=A16, ws=A16, ws_bytes=256,
+             cs=[32768])
+    a.update(kw)
+    cs = (ctypes.c_int32 * len(a["cs"]))(*a["cs"])
+    return lib.ca_chunk_attention(a["Q"], a["K"], a["V"], a["tables"], a["counts"], cs, a["B"],
+                                  a["H_q"], a["H_kv"], a["C"], a["L_max"], a["D"], a["blk"],
+                                  a["scale"], a["O"], a["LSE"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Q=None), ca.CA_ERR_INVALID_ARG),
+    (dict(tables=None), ca.CA_ERR_INVALID_ARG),
+    (dict(ws=None), ca.CA_ERR_INVALID_ARG),
+    (dict(C=0), ca.CA_ERR_INVALID_ARG),
+    (dict(scale=0.0), ca.CA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), ca.CA_ERR_INVALID_ARG),
+    (dict(H_kv=6), ca.CA_ERR_SHAPE),
+    (dict(L_max=34800), ca.CA_ERR_SHAPE),
+    (dict(cs=[33000]), ca.CA_ERR_SHAPE),
+    (dict(cs=[-1]), ca.CA_ERR_SHAPE),
+    (dict(D=96), ca.CA_ERR_UNSUPPORTED),
+    (dict(blk=32, L_max=34816), ca.CA_ERR_UNSUPPORTED),
+    (dict(H_q=96, H_kv=3), ca.CA_ERR_UNSUPPORTED),
+    (dict(Q=A_MIS), ca.CA_ERR_ALIGN),
+    (dict(O=A_MIS), ca.CA_ERR_ALIGN),
+    (dict(ws_bytes=16), ca.CA_ERR_WORKSPACE),
+    (dict(ws=ctypes.c_void_p((1 << 20) + 16)), ca.CA_ERR_WORKSPACE),
+])
+def test_attention_host_checks(lib, kw, code):
+    assert _attn(lib, **kw) == code
+
+
+def test_dense_host_checks(lib):
+    cs = (ctypes.c_int32 * 1)(32768)
+    st = lib.ca_dense_chunk_attention(A16, A16, A16, cs, 1, 32, 8, 2048, 34816, 96, 128, 0.1,
+                                      A16, A16, A16, 256, None)
+    assert st == ca.CA_ERR_UNSUPPORTED
+    st = lib.ca_dense_chunk_attention(A16, A16, A16, None, 1, 32, 8, 2048, 34816, 128, 128, 0.1,
+                                      A16, A16, A16, 256, None)
+    assert st == ca.CA_ERR_INVALID_ARG
+
+
+def test_build_tables_host_checks(lib):
+    f = lib.ca_build_block_tables
+    assert f(None, 1, 32, 16, 272, 4, A16, A16, None, None, None) == ca.CA_ERR_INVALID_ARG
+    assert f(A16, 1, 32, 16, 272, 5, A16, A16, None, None, None) == ca.CA_ERR_SHAPE
+    assert f(A16, 1, 32, 16, 272, 4, A_MIS, A16, None, None, None) == ca.CA_ERR_ALIGN
+    assert f(A16, 1, 32, 16, 272, 4, A16, A16, None, A16, None) == ca.CA_ERR_INVALID_ARG
+    assert f(A16, 0, 32, 16, 272, 4, A16, A16, None, None, None) == ca.CA_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    import importlib
+    monkeypatch.setattr(ca, "_lib", None)
+    monkeypatch.setattr(ca, "_LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError):
+        ca.load_library()

@@ -1,0 +1,83 @@
+"""Block-Union table construction on the GPU vs the CPU oracle: bit-exact
+tables (padding included), counts and CSR on every workload and on edge
+cases (odd widths that take the scalar path, misaligned masks, empty and full
+masks, nonzero values other than 1, every supported group size)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import serving_block_union_b200 as ca
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+WORKLOADS = ["tiny", "llama8b_32k", "llama8b_128k_d2", "llama8b_128k_d5", "llama8b_128k_d10",
+             "llama8b_128k_d20", "llama8b_128k_noise", "batched", "full_prefill_c0",
+             "full_prefill_c1", "full_prefill_c31", "full_prefill_c63"]
+
+
+def _check(mask_np, group, mask_dev=None):
+    T_ref, c_ref, ip_ref, ix_ref = oracle.block_tables(mask_np, group)
+    m = mask_dev if mask_dev is not None else torch.from_numpy(mask_np).cuda()
+    T, c, ip, ix = ca.build_block_tables(m, group, csr=True)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(T.cpu().numpy(), T_ref)
+    np.testing.assert_array_equal(c.cpu().numpy(), c_ref)
+    np.testing.assert_array_equal(ip.cpu().numpy(), ip_ref)
+    n = int(ip_ref[-1])
+    np.testing.assert_array_equal(ix.cpu().numpy()[:n], ix_ref)
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_tables_bit_exact_on_workloads(cuda_ok, name):
+    wl = workloads.by_name(name)
+    _check(workloads.make_mask(wl), wl.group)
+
+
+@pytest.mark.parametrize("shape", [
+    # B, H_q, nQ, nKVmax, G
+    (1, 4, 4, 16, 4), (2, 8, 3, 37, 2), (3, 6, 5, 50, 3), (1, 8, 1, 9, 8),
+    (2, 4, 2, 7, 1), (1, 32, 16, 16400, 4), (1, 2, 64, 3000, 2), (5, 16, 2, 1, 16),
+])
+@pytest.mark.parametrize("p", [0.0, 0.01, 0.3, 1.0])
+def test_tables_random_shapes(cuda_ok, shape, p):
+    B, H_q, nQ, nK, G = shape
+    rng = np.random.default_rng(abs(hash((shape, p))) % 2**32)
+    mask = (rng.random((B, H_q, nQ, nK)) < p).astype(np.uint8)
+    mask[mask == 1] = rng.integers(1, 256, size=int(mask.sum()), dtype=np.uint8)
+    _check(mask, G)
+
+
+def test_tables_misaligned_mask_pointer(cuda_ok):
+    rng = np.random.default_rng(5)
+    B, H_q, nQ, nK, G = 2, 8, 4, 64, 4
+    mask = (rng.random((B, H_q, nQ, nK)) < 0.05).astype(np.uint8)
+    flat = torch.zeros(mask.size + 1, dtype=torch.uint8, device="cuda")
+    view = flat[1:].view(B, H_q, nQ, nK)
+    view.copy_(torch.from_numpy(mask))
+    _check(mask, G, mask_dev=view)
+
+
+def test_tables_bool_mask(cuda_ok):
+    rng = np.random.default_rng(9)
+    mask = rng.random((1, 8, 4, 48)) < 0.1
+    T_ref, c_ref, _, _ = oracle.block_tables(mask.astype(np.uint8), 2)
+    T, c, _, _ = ca.build_block_tables(torch.from_numpy(mask).cuda(), 2)
+    np.testing.assert_array_equal(T.cpu().numpy(), T_ref)
+    np.testing.assert_array_equal(c.cpu().numpy(), c_ref)
+
+
+def test_tables_stream_ordering(cuda_ok):
+    """Launch on a side stream; results visible after that stream syncs."""
+    wl = workloads.llama8b_32k()
+    mask = workloads.make_mask(wl)
+    s = torch.cuda.Stream()
+    m = torch.from_numpy(mask).cuda()
+    torch.cuda.current_stream().synchronize()
+    with torch.cuda.stream(s):
+        T, c, _, _ = ca.build_block_tables(m, wl.group, stream=s)
+    s.synchronize()
+    T_ref, c_ref, _, _ = oracle.block_tables(mask, wl.group)
+    np.testing.assert_array_equal(T.cpu().numpy(), T_ref)
+    np.testing.assert_array_equal(c.cpu().numpy(), c_ref)
