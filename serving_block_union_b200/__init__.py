@@ -39,7 +39,8 @@ __all__ = [
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "libcompactattn.so")
+# CA_LIBRARY selects another build of the library (e.g. a tuning variant)
+_LIB_PATH = os.environ.get("CA_LIBRARY") or os.path.join(_HERE, "libcompactattn.so")
 _lock = threading.Lock()
 _lib = None
 

@@ -46,14 +46,39 @@ namespace ca {
 namespace {
 
 constexpr int kTileM = 128;
-constexpr int kThreads = 320;
+// Three warpgroups: two softmax warpgroups (one per tile) and one for the MMA
+// issuer (warp 8), the TMA producer (warp 9) and two idle warps. Launched at
+// kLaunchRegs registers per thread; the softmax warpgroups then grow to
+// kSoftmaxRegs and the third shrinks to kControlRegs:
+// 2 * 128 * 224 + 128 * 56 = 384 * 168, and per SM sub-partition (one warp of
+// each warpgroup) 224 + 224 + 56 = 3 * 168.
+#ifndef CA_REG_SPLIT
+#define CA_REG_SPLIT 0
+#endif
+constexpr bool kRegSplit = CA_REG_SPLIT != 0;
+constexpr int kThreads = kRegSplit ? 384 : 320;
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
+constexpr int kLaunchRegs = 168;
+#ifndef CA_SOFTMAX_REGS
+#define CA_SOFTMAX_REGS 224
+#endif
+constexpr int kSoftmaxRegs = CA_SOFTMAX_REGS;
+constexpr int kControlRegs = 3 * kLaunchRegs - 2 * kSoftmaxRegs;
+static_assert(2 * kSoftmaxRegs + kControlRegs == 3 * kLaunchRegs, "register split must balance");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr int kSmemBudget = 227 * 1024;
 constexpr int kSmemFloor = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
+
+// Keys per P chunk handed from the softmax to the P.V MMA (32, 64 or 128).
+#ifndef CA_P_CHUNK_KEYS
+#define CA_P_CHUNK_KEYS 64
+#endif
+constexpr int kPChunkKeysCfg = CA_P_CHUNK_KEYS;
+static_assert(kPChunkKeysCfg == 32 || kPChunkKeysCfg == 64 || kPChunkKeysCfg == 128,
+              "P chunk must be 32, 64 or 128 keys");
 
 struct Params {
     int B, H_q, H_kv, C, L_max, G, R, n_pairs, nKVmax;
@@ -77,7 +102,9 @@ struct Layout {
     static constexpr int kKOff = 2 * kQTile;
     static constexpr int kVOff = kKOff + kStages * kKV;
     static constexpr int kBarOff = kVOff + kStages * kKV;
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1;
+    static constexpr int kPChunkKeys = kPChunkKeysCfg < BLK ? kPChunkKeysCfg : BLK;
+    static constexpr int kPChunks = BLK / kPChunkKeys;  // P reaches the MMA chunk by chunk
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 * kPChunks + 2 + 1;
     static constexpr int kEnd = kBarOff + kNumBars * 8 + 16;
     static constexpr int kDynamic = (kEnd + 1024) > kSmemFloor ? (kEnd + 1024) : kSmemFloor;
     static_assert(kStages >= 2, "need at least two K/V stages");
@@ -99,6 +126,29 @@ __device__ __forceinline__ int count_le(const int32_t *T, int n, int bound, int 
         hi = lo;
     }
     return 0;
+}
+
+// Share of the softmax exponentials evaluated by the FMA-pipe polynomial
+// (exp2_poly) instead of the MUFU unit: column c uses it when
+// c % kPolyEvery == kPolyEvery - 1 (0 disables it).
+#ifndef CA_POLY_EVERY
+#define CA_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = CA_POLY_EVERY;
+
+__device__ __forceinline__ constexpr bool use_poly(int c) {
+    return kPolyEvery > 0 && (c % kPolyEvery) == kPolyEvery - 1;
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, uint32_t (&r)[N]);
+template <>
+__device__ __forceinline__ void tmem_ld_row<128>(uint32_t taddr, uint32_t (&r)[128]) {
+    tmem_ld128(taddr, r);
+}
+template <>
+__device__ __forceinline__ void tmem_ld_row<64>(uint32_t taddr, uint32_t (&r)[64]) {
+    tmem_ld64(taddr, r);
 }
 
 template <int D, int BLK, bool DENSE>
@@ -123,9 +173,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *k_empty = k_full + NST;
     uint64_t *v_full = k_empty + NST;
     uint64_t *v_empty = v_full + NST;
-    uint64_t *s_full = v_empty + NST;  // [2]
-    uint64_t *p_full = s_full + 2;     // [2]
-    uint64_t *o_full = p_full + 2;     // [2]
+    constexpr int NPC = L::kPChunks;
+    uint64_t *s_full = v_empty + NST;   // [2]
+    uint64_t *p_full = s_full + 2;      // [2][NPC]: P chunk c of tile t stored in TMEM
+    uint64_t *o_full = p_full + 2 * NPC;  // [2]
     uint64_t *mma_done = o_full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
@@ -158,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(s_full + t, 1);
-            mbar_init(p_full + t, 4);
+            for (int c = 0; c < NPC; ++c) mbar_init(p_full + t * NPC + c, 4);
             mbar_init(o_full + t, 1);
         }
         mbar_init(mma_done, 1);
@@ -197,7 +248,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         n_full = count_le(T, n_eff, jfull, lane);
     }
 
-    if (warp == kTmaWarp) {
+    // Role code sits inside the branch that re-sized its registers, so the
+    // compiler allocates each role within its own budget.
+    if (warp >= kMmaWarp) {
+      if (kRegSplit) regs_dec<kControlRegs>();
+      if (warp == kTmaWarp) {
         // ================================================================ producer
         int k_issued = 0, v_issued = 0;  // loads started (for the drain below)
         bool q_issued = false;
@@ -271,28 +326,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == kMmaWarp) {
         // ================================================================ MMA issue
         if (n_eff > 0 && lane == 0) {
-            const uint32_t q_addr = sbase + L::kQOff;
-            const uint32_t k_addr = sbase + L::kKOff;
-            const uint32_t v_addr = sbase + L::kVOff;
+            // Descriptors: the high words are constant; the low words of the Q
+            // tiles are fixed for the item and those of a K / V stage are a base
+            // plus the stage offset, so each MMA costs one add and the issue.
+            const uint64_t dq = sdesc_sw128(sbase + L::kQOff, 16, 1024);
+            const uint64_t dk = sdesc_sw128(sbase + L::kKOff, 16, 1024);
+            const uint64_t dv = sdesc_sw128(sbase + L::kVOff, BLK * 128, 1024);
+            const uint32_t q_lo = static_cast<uint32_t>(dq), q_hi = static_cast<uint32_t>(dq >> 32);
+            const uint32_t k_lo = static_cast<uint32_t>(dk), k_hi = static_cast<uint32_t>(dk >> 32);
+            const uint32_t v_lo = static_cast<uint32_t>(dv), v_hi = static_cast<uint32_t>(dv >> 32);
+            constexpr uint32_t kStageUnits = L::kKV >> 4;  // one stage, in descriptor units
             auto issue_s = [&](int t, int slot) {
+                const uint32_t a0 = q_lo + t * (L::kQTile >> 4);
+                const uint32_t b0 = k_lo + slot * kStageUnits;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk & 3) * 32;  // 16 bf16 = 32 B inside the swizzle row
-                    const uint64_t a = sdesc_sw128(
-                        q_addr + t * L::kQTile + (kk >> 2) * (kTileM * 128) + off, 16, 1024);
-                    const uint64_t bb = sdesc_sw128(
-                        k_addr + slot * L::kKV + (kk >> 2) * (BLK * 128) + off, 16, 1024);
-                    mma_ss(tmem + t * 128, a, bb, kIdescS, kk > 0 ? 1u : 0u);
+                    // 16 bf16 = 32 B steps inside a 128-B swizzle row; a new 64-column
+                    // sub-tile every 4 steps
+                    const uint32_t ao = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
+                    const uint32_t bo = ((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4;
+                    mma_ss_w(tmem + t * 128, a0 + ao, q_hi, b0 + bo, k_hi, kIdescS,
+                             kk > 0 ? 1u : 0u);
                 }
             };
-            auto issue_pv = [&](int t, int slot, bool acc) {
+            // P.V of tile t, chunk by chunk as the softmax hands P over; false if a
+            // wait gave up.
+            auto issue_pv = [&](int t, int slot, bool acc, uint32_t par) -> bool {
+                const uint32_t b0 = v_lo + slot * kStageUnits;
 #pragma unroll
-                for (int kk = 0; kk < BLK / 16; ++kk) {
-                    const uint64_t bb =
-                        sdesc_sw128(v_addr + slot * L::kKV + kk * (16 * 128), BLK * 128, 1024);
-                    mma_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, bb, kIdescPV,
-                           (acc || kk > 0) ? 1u : 0u);
+                for (int c = 0; c < NPC; ++c) {
+                    if (!mbar_wait(p_full + t * NPC + c, par, ab)) return false;
+                    tc_fence_after();
+                    constexpr int KPC = L::kPChunkKeys / 16;  // MMAs (K = 16) per chunk
+#pragma unroll
+                    for (int kk = KPC * c; kk < KPC * c + KPC; ++kk) {
+                        mma_ts_w(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                                 b0 + ((kk * (16 * 128)) >> 4), v_hi, kIdescPV,
+                                 (acc || kk > 0) ? 1u : 0u);
+                    }
                 }
+                return true;
             };
             bool ok = mbar_wait(q_full, 0, ab) && mbar_wait(k_full, 0, ab);
             if (ok) {
@@ -310,9 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int s1 = (j + 1) % NST;
                 const uint32_t ph1 = ((j + 1) / NST) & 1;
                 if (!(ok = mbar_wait(v_full + s, ph, ab))) break;
-                if (!(ok = mbar_wait(p_full + 0, j & 1, ab))) break;
-                tc_fence_after();
-                issue_pv(0, s, j > 0);
+                if (!(ok = issue_pv(0, s, j > 0, j & 1))) break;
                 if (more) {
                     if (!(ok = mbar_wait(k_full + s1, ph1, ab))) break;
                     tc_fence_after();
@@ -321,9 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 } else {
                     tc_commit(o_full + 0);
                 }
-                if (!(ok = mbar_wait(p_full + 1, j & 1, ab))) break;
-                tc_fence_after();
-                issue_pv(1, s, j > 0);
+                if (!(ok = issue_pv(1, s, j > 0, j & 1))) break;
                 tc_commit(v_empty + s);
                 if (more) {
                     issue_s(1, s1);
@@ -338,7 +407,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait_drain(mma_done, 0);
         }
         __syncwarp();
+      }
     } else {
+        if (kRegSplit) regs_inc<kSoftmaxRegs>();
         // ================================================================ softmax
         const int t = warp >> 2;
         const int qw = warp & 3;
@@ -363,12 +434,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             float s[BLK];
+            {
+                uint32_t v[BLK];
+                tmem_ld_row<BLK>(tS, v);  // the whole S row in one TMEM round trip
 #pragma unroll
-            for (int c = 0; c < BLK / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld32(tS + c * 32, v);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(v[i]);
+                for (int i = 0; i < BLK; ++i) s[i] = __uint_as_float(v[i]);
             }
             if (j >= n_full) {
                 int jb = DENSE ? j : __ldg(T + j);
@@ -378,10 +448,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < BLK; ++c)
                     if (c > lim) s[c] = -INFINITY;
             }
-            float mx = s[0];
+            // row max: 8 independent chains of 3-input max, then a short tree
+            float mx8[8];
 #pragma unroll
-            for (int c = 1; c < BLK; ++c) mx = fmaxf(mx, s[c]);
-            const float m_blk = mx * sl2;
+            for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+#pragma unroll
+            for (int c = 8; c + 8 < BLK; c += 16)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], s[c + k], s[c + 8 + k]);
+            if ((BLK - 8) % 16 != 0) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], s[BLK - 8 + k]);
+            }
+            const float m_blk = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
+                                      fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7])) * sl2;
             const float m_new = fmaxf(m_run, m_blk);
             const bool old_finite = m_run != -INFINITY;
             const bool upd = old_finite ? (m_new > m_run + kRescaleThreshold)
@@ -391,40 +471,54 @@ __global__ void __launch_bounds__(kThreads, 1)
                 alpha = old_finite ? ex2_approx(m_run - m_new) : 0.0f;
                 m_run = m_new;
             }
-            const float m_use = m_run == -INFINITY ? 0.0f : m_run;
-            l_run *= alpha;
-            float sum = 0.0f;
-#pragma unroll
-            for (int c = 0; c < BLK / 64; ++c) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float p0 = ex2_approx(fmaf(s[c * 64 + 2 * i], sl2, -m_use));
-                    const float p1 = ex2_approx(fmaf(s[c * 64 + 2 * i + 1], sl2, -m_use));
-                    sum += p0 + p1;
-                    pk[i] = pack_bf16x2(p0, p1);
-                }
-                tmem_st32(tS + c * 32, pk);
-            }
-            l_run += sum;
             // O rescale (rare: only when a row's max grew past the threshold). O is
-            // stable here: S(j) was committed after P.V(j-1) was issued.
+            // stable here: S(j) was committed after P.V(j-1) was issued. It must land
+            // before the first P chunk is handed over.
             const bool need = upd && old_finite && j > 0;
             if (__any_sync(0xffffffffu, need)) {
                 const float a = need ? alpha : 1.0f;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t v[32];
-                    tmem_ld32(tO + c * 32, v);
+                for (int c = 0; c < D / 16; ++c) {
+                    uint32_t v[16];
+                    tmem_ld16(tO + c * 16, v);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
-                    tmem_st32(tO + c * 32, v);
+                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
+                    tmem_st16(tO + c * 16, v);
                 }
             }
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(p_full + t);
+            const float m_use = m_run == -INFINITY ? 0.0f : m_run;
+            l_run *= alpha;
+            float acc[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = 0.0f;
+#pragma unroll
+            for (int c = 0; c < NPC; ++c) {
+                constexpr int CK = L::kPChunkKeys;
+                uint32_t pk[CK / 2];
+#pragma unroll
+                for (int i = 0; i < CK / 2; ++i) {
+                    const int e0 = c * CK + 2 * i;
+                    const float x0 = fmaf(s[e0], sl2, -m_use);
+                    const float x1 = fmaf(s[e0 + 1], sl2, -m_use);
+                    const float p0 = use_poly(e0) ? exp2_poly(x0) : ex2_approx(x0);
+                    const float p1 = use_poly(e0 + 1) ? exp2_poly(x1) : ex2_approx(x1);
+                    acc[(2 * i) & 7] += p0;
+                    acc[(2 * i + 1) & 7] += p1;
+                    pk[i] = pack_bf16x2(p0, p1);
+                }
+#pragma unroll
+                for (int q = 0; q < CK / 32; ++q) tmem_st16(tS + c * (CK / 2) + q * 16, pk + q * 16);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                mbar_arrive_lane0(p_full + t * NPC + c, lane);
+            }
+#pragma unroll
+            for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+                for (int k = 0; k < w; ++k) acc[k] += acc[k + w];
+            const float sum = acc[0];
+            l_run += sum;
         }
         bool have_o = false;
         if (n_eff > 0 && __all_sync(0xffffffffu, ok)) {
@@ -510,6 +604,16 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
                                         L::kDynamic);
     });
     if (attr_err != cudaSuccess) return CA_ERR_CUDA;
+    // The in-kernel register split assumes exactly kLaunchRegs registers per
+    // thread at launch; any other count could leave a warpgroup waiting for
+    // registers that never come, so refuse to launch instead.
+    static int num_regs = -1;
+    if (num_regs < 0) {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return CA_ERR_CUDA;
+        num_regs = fa.numRegs;
+    }
+    if (kRegSplit && num_regs != kLaunchRegs) return CA_ERR_UNSUPPORTED;
 
     const int G = a.H_q / a.H_kv;
     const int R = kTileM / G;
