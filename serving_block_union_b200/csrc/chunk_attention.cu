@@ -15,14 +15,23 @@
 //   n_eff  = #{t : T[t] <= last position / blk}          (later blocks unread)
 //   n_full = #{t : T[t] <= (first position + 1) / blk - 1} (no causal mask)
 //
-// Warp roles (320 threads, one CTA per SM):
+// Grid: one CTA per item, items ordered so that the CTAs resident together
+// cover a few tile pairs of every group and start the group's table at the
+// same time: they walk its blocks in lockstep, each block comes from HBM once
+// and then from L2. (A persistent stream-K schedule that balances the last
+// wave staggers the CTAs instead and read several times more DRAM; under the
+// 1 kW power cap that sustained runs reach, it was not faster either.)
+//
+// Warp roles (384 threads, one CTA per SM):
 //   warps 0-3  softmax + epilogue of tile 0 (thread = TMEM lane = packed row)
 //   warps 4-7  softmax + epilogue of tile 1
 //   warp 8     MMA issue (one elected lane) + TMEM allocation
 //   warp 9     TMA producer (Q once, then K and V of T[0..n_eff) in a ring)
+//   warps 10-11 idle (they complete the third warpgroup of the register split)
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,384) O1 [384,512);
 // P (bf16 pairs) overwrites the first blk/2 columns of S and feeds the P.V MMA
-// straight from tensor memory.
+// straight from tensor memory, in chunks of 64 keys as the softmax produces
+// them.
 // MMA order per block j: PV0(j), S0(j+1), PV1(j), S1(j+1): while tile 0's
 // softmax works on S0(j+1) the tensor core runs tile 1's products and the
 // other way round.
@@ -46,14 +55,16 @@ namespace ca {
 namespace {
 
 constexpr int kTileM = 128;
-// Three warpgroups: two softmax warpgroups (one per tile) and one for the MMA
-// issuer (warp 8), the TMA producer (warp 9) and two idle warps. Launched at
-// kLaunchRegs registers per thread; the softmax warpgroups then grow to
-// kSoftmaxRegs and the third shrinks to kControlRegs:
-// 2 * 128 * 224 + 128 * 56 = 384 * 168, and per SM sub-partition (one warp of
-// each warpgroup) 224 + 224 + 56 = 3 * 168.
+// Register split (setmaxnreg): three warpgroups — two softmax warpgroups (one
+// per tile) and one holding the MMA issuer, the TMA producer and two idle
+// warps. Launched at kLaunchRegs registers per thread (the most 384 threads
+// can have: three warps share each SM sub-partition's 16K registers); the
+// softmax warpgroups then grow to kSoftmaxRegs and the third shrinks to
+// kControlRegs, so that per sub-partition (one warp of each warpgroup)
+// 2 * kSoftmaxRegs + kControlRegs = 3 * kLaunchRegs (208 + 208 + 88 = 504).
+// Without the split (CA_REG_SPLIT=0) the kernel runs 320 threads at 168.
 #ifndef CA_REG_SPLIT
-#define CA_REG_SPLIT 0
+#define CA_REG_SPLIT 1
 #endif
 constexpr bool kRegSplit = CA_REG_SPLIT != 0;
 constexpr int kThreads = kRegSplit ? 384 : 320;
@@ -61,11 +72,13 @@ constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
 constexpr int kLaunchRegs = 168;
 #ifndef CA_SOFTMAX_REGS
-#define CA_SOFTMAX_REGS 224
+#define CA_SOFTMAX_REGS 208
 #endif
 constexpr int kSoftmaxRegs = CA_SOFTMAX_REGS;
 constexpr int kControlRegs = 3 * kLaunchRegs - 2 * kSoftmaxRegs;
 static_assert(2 * kSoftmaxRegs + kControlRegs == 3 * kLaunchRegs, "register split must balance");
+static_assert(kSoftmaxRegs % 8 == 0 && kControlRegs % 8 == 0 && kControlRegs >= 24,
+              "setmaxnreg counts are multiples of 8, at least 24");
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.693147180559945309f;
@@ -129,15 +142,16 @@ __device__ __forceinline__ int count_le(const int32_t *T, int n, int bound, int 
 }
 
 // Share of the softmax exponentials evaluated by the FMA-pipe polynomial
-// (exp2_poly) instead of the MUFU unit: column c uses it when
-// c % kPolyEvery == kPolyEvery - 1 (0 disables it).
+// (exp2_poly2) instead of the MUFU unit, in pairs of columns.
 #ifndef CA_POLY_EVERY
 #define CA_POLY_EVERY 0
 #endif
 constexpr int kPolyEvery = CA_POLY_EVERY;
 
-__device__ __forceinline__ constexpr bool use_poly(int c) {
-    return kPolyEvery > 0 && (c % kPolyEvery) == kPolyEvery - 1;
+// Pair q (columns 2q, 2q+1) of an S row goes to the FMA-pipe polynomial when
+// q % kPolyEvery == kPolyEvery - 1 (0 disables it).
+__device__ __forceinline__ constexpr bool use_poly_pair(int q) {
+    return kPolyEvery > 0 && (q % kPolyEvery) == kPolyEvery - 1;
 }
 
 template <int N>
@@ -488,9 +502,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float m_use = m_run == -INFINITY ? 0.0f : m_run;
             l_run *= alpha;
-            float acc[8];
+            // exponentials in pairs: x = s * scale_log2 - m as one f32x2 FMA, the
+            // row sum in four f32x2 accumulators; the MUFU unit does most pairs,
+            // the FMA pipe the pairs use_poly_pair() selects
+            const uint64_t sl2x2 = f2_pack(sl2, sl2);
+            const uint64_t nm2 = f2_pack(-m_use, -m_use);
+            uint64_t acc2[4];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) acc[k] = 0.0f;
+            for (int k = 0; k < 4; ++k) acc2[k] = 0ull;
 #pragma unroll
             for (int c = 0; c < NPC; ++c) {
                 constexpr int CK = L::kPChunkKeys;
@@ -498,13 +517,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < CK / 2; ++i) {
                     const int e0 = c * CK + 2 * i;
-                    const float x0 = fmaf(s[e0], sl2, -m_use);
-                    const float x1 = fmaf(s[e0 + 1], sl2, -m_use);
-                    const float p0 = use_poly(e0) ? exp2_poly(x0) : ex2_approx(x0);
-                    const float p1 = use_poly(e0 + 1) ? exp2_poly(x1) : ex2_approx(x1);
-                    acc[(2 * i) & 7] += p0;
-                    acc[(2 * i + 1) & 7] += p1;
-                    pk[i] = pack_bf16x2(p0, p1);
+                    const uint64_t x2 = f2_fma(f2_pack(s[e0], s[e0 + 1]), sl2x2, nm2);
+                    const uint64_t p2 = use_poly_pair(e0 / 2)
+                                            ? exp2_poly2(x2)
+                                            : f2_pack(ex2_approx(f2_lo(x2)), ex2_approx(f2_hi(x2)));
+                    acc2[i & 3] = f2_add(acc2[i & 3], p2);
+                    pk[i] = pack_bf16x2(f2_lo(p2), f2_hi(p2));
                 }
 #pragma unroll
                 for (int q = 0; q < CK / 32; ++q) tmem_st16(tS + c * (CK / 2) + q * 16, pk + q * 16);
@@ -513,11 +531,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 mbar_arrive_lane0(p_full + t * NPC + c, lane);
             }
-#pragma unroll
-            for (int w = 4; w > 0; w >>= 1)
-#pragma unroll
-                for (int k = 0; k < w; ++k) acc[k] += acc[k + w];
-            const float sum = acc[0];
+            acc2[0] = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
+            const float sum = f2_lo(acc2[0]) + f2_hi(acc2[0]);
             l_run += sum;
         }
         bool have_o = false;

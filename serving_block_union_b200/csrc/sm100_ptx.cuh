@@ -395,6 +395,47 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
+// ---- packed fp32 pairs (sm_100 f32x2 arithmetic: two lanes per instruction)
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) {
+    return __uint_as_float(static_cast<uint32_t>(v));
+}
+__device__ __forceinline__ float f2_hi(uint64_t v) {
+    return __uint_as_float(static_cast<uint32_t>(v >> 32));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// exp2_poly on a pair, with the pair arithmetic in f32x2 form (same method,
+// same coefficients and the same -127 clamp as exp2_poly above).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+    const uint64_t xc = f2_pack(fmaxf(f2_lo(x2), -127.0f), fmaxf(f2_hi(x2), -127.0f));
+    const uint64_t kRound2 = f2_pack(12582912.0f, 12582912.0f);
+    const uint64_t t = f2_add(xc, kRound2);
+    const uint64_t r = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
+    const uint64_t f = f2_fma(r, f2_pack(-1.0f, -1.0f), xc);
+    uint64_t p = f2_fma(f2_pack(0.055009059607982635f, 0.055009059607982635f), f,
+                        f2_pack(0.2422109693288803f, 0.2422109693288803f));
+    p = f2_fma(p, f, f2_pack(0.6932829022407532f, 0.6932829022407532f));
+    p = f2_fma(p, f, f2_pack(1.0f, 1.0f));
+    const uint32_t lo = __float_as_uint(f2_lo(t)) * 8388608u + __float_as_uint(f2_lo(p));
+    const uint32_t hi = __float_as_uint(f2_hi(t)) * 8388608u + __float_as_uint(f2_hi(p));
+    return f2_pack(__uint_as_float(lo), __uint_as_float(hi));
+}
+
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
