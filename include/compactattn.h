@@ -131,6 +131,32 @@ int ca_dense_chunk_attention(const void *Q, const void *K, const void *V,
                              int L_max, int D, int blk, float scale, void *O, float *LSE,
                              void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * ca_chunk_attention without a caller workspace, for callers that cannot
+ * allocate device memory when they run attention (an engine whose device
+ * memory is sized once at start-up, code inside a fixed memory pool, a host
+ * path that must not enter the allocator). The paper has no counterpart: this
+ * is a deployment convenience of this library.
+ *
+ * Same arguments and results as ca_chunk_attention minus the workspace; it
+ * allocates nothing (no cudaMalloc / cudaFree, no allocating library call).
+ * The scratch it needs comes from a fixed 4096-byte array inside the library,
+ * held by every GPU that loads the library until the process exits; sizes whose
+ * workspace (ca_workspace_bytes) would exceed it return CA_ERR_WORKSPACE.
+ * The first call on each device looks up that device's copy of the array
+ * (cudaGetSymbolAddress, with that device current), so make that first call
+ * before any stream capture. Every call on a device shares the one array:
+ * calls that overlap on the GPU (for example on two streams at once) race, so
+ * serialise them. Each call clears the device status word first; if
+ * device_status (a device pointer to one uint32, or NULL) is given, the call
+ * copies the final status word there on the same stream: bit 0 set = an
+ * invalid table or count was found, bit 1 set = a bounded wait expired.
+ */
+int ca_chunk_attention_noalloc(const void *Q, const void *K, const void *V, const int32_t *tables,
+                               const int32_t *counts, const int32_t *chunk_start, int B, int H_q,
+                               int H_kv, int C, int L_max, int D, int blk, float scale, void *O,
+                               float *LSE, unsigned int *device_status, void *stream);
+
 /* Synchronises `stream`, then reads the workspace status word written by the
  * kernels: CA_OK, CA_ERR_TABLE or CA_ERR_TIMEOUT (sticky until the workspace is
  * zeroed again; CA_ERR_TABLE wins if both are set). CA_ERR_CUDA if the stream

@@ -35,6 +35,7 @@ __all__ = [
     "chunk_attention",
     "dense_chunk_attention",
     "read_device_status",
+    "chunk_attention_noalloc",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -62,6 +63,7 @@ EXPORTED_SYMBOLS = (
     "ca_chunk_attention",
     "ca_dense_chunk_attention",
     "ca_read_device_status",
+    "ca_chunk_attention_noalloc",
 )
 
 
@@ -100,6 +102,9 @@ def load_library():
         lib.ca_dense_chunk_attention.restype = I
         lib.ca_read_device_status.argtypes = [P, P]
         lib.ca_read_device_status.restype = I
+        lib.ca_chunk_attention_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P, P,
+                                                   P, P]
+        lib.ca_chunk_attention_noalloc.restype = I
         _lib = lib
         return lib
 
@@ -276,3 +281,45 @@ def read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stre
     CA_ERR_TIMEOUT)."""
     return int(load_library().ca_read_device_status(_ptr(workspace),
                                                       _stream_handle(stream, workspace.device)))
+
+
+def chunk_attention_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                            tables: torch.Tensor, counts: torch.Tensor,
+                            chunk_start: Sequence[int], O: torch.Tensor, LSE: torch.Tensor,
+                            scale: Optional[float] = None,
+                            device_status: Optional[torch.Tensor] = None,
+                            stream: Optional[torch.cuda.Stream] = None
+                            ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """chunk_attention for callers that cannot allocate device memory: no
+    workspace, and the caller passes the outputs O and LSE (this wrapper
+    allocates nothing either). The library's fixed scratch array stands in for
+    the workspace; calls that overlap on the GPU share it and race.
+    ``device_status``: optional int32 CUDA tensor of one element that receives
+    the call's device status word (0 = OK)."""
+    _need(tables, "tables", torch.int32, 3)
+    _need(counts, "counts", torch.int32, 2)
+    _need(Q, "Q", torch.bfloat16, 4)
+    _need(K, "K", torch.bfloat16, 4)
+    _need(V, "V", torch.bfloat16, 4)
+    _need(O, "O", torch.bfloat16, 4)
+    _need(LSE, "LSE", torch.float32, 3)
+    B, H_q, C, D = Q.shape
+    _, H_kv, L_max, _ = K.shape
+    nK = tables.shape[-1]
+    if nK <= 0 or L_max % nK:
+        raise ValueError("tables' last dim must divide L_max (it is L_max / blk)")
+    if tuple(O.shape) != tuple(Q.shape) or tuple(LSE.shape) != (B, H_q, C):
+        raise ValueError("O must have Q's shape and LSE [B, H_q, C]")
+    if device_status is not None:
+        if (device_status.dtype != torch.int32 or not device_status.is_cuda
+                or device_status.numel() < 1):
+            raise ValueError("device_status must be an int32 CUDA tensor of one element")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    cs = _chunk_start_host(chunk_start, B)
+    st = load_library().ca_chunk_attention_noalloc(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(tables), _ptr(counts), cs, B, H_q, H_kv, C, L_max, D,
+        L_max // nK, float(scale), _ptr(O), _ptr(LSE), _ptr(device_status),
+        _stream_handle(stream, Q.device))
+    _check("ca_chunk_attention_noalloc", st)
+    return O, LSE
