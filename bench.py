@@ -202,7 +202,7 @@ def oracle_sample_rate(wl, mask, Q, K, V, target_s: float = 15.0, max_rows: int 
     return flops / dt / 1e12, int(rows.size), dt, threads
 
 
-def run_reference(args, wl):
+def run_reference(args, wl, name=None):
     import workloads
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -225,7 +225,7 @@ def run_reference(args, wl):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": secs * 1e3 / max(1, args.steps), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": _config(wl),
+        "config": _config(wl, name),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -235,18 +235,40 @@ def run_reference(args, wl):
     return 0
 
 
-def _config(wl):
-    return {"workload": wl.name, "B": wl.B, "H_q": wl.H_q, "H_kv": wl.H_kv, "D": wl.D,
-            "block": wl.blk, "chunk": wl.C, "cached_tokens": list(wl.chunk_start),
-            "mask_density": wl.density if wl.density else None,
-            "l2": "256 MB L2 flush between timed steps; K/V cache larger than L2"}
+def _config(wl, name=None, n_chunks=1):
+    cfg = {"workload": name or wl.name, "B": wl.B, "H_q": wl.H_q, "H_kv": wl.H_kv, "D": wl.D,
+           "block": wl.blk, "chunk": wl.C, "cached_tokens": list(wl.chunk_start),
+           "mask_density": wl.density if wl.density else None,
+           "l2": "256 MB L2 flush between timed steps; K/V cache larger than L2"}
+    if n_chunks > 1:
+        cfg["chunks_per_step"] = n_chunks
+        cfg["cached_tokens"] = f"0..{wl.chunk_start[0]} (chunk k starts at {wl.C}*k)"
+    return cfg
+
+
+def max_over_ranks(t, world: int) -> float:
+    """Max of a one-element tensor over all ranks (the job's time is its
+    slowest rank's); world 1 returns the value."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
 
-def run_ours(args, wl):
+def step_chunks(name: str):
+    """Workloads of the chunks one step processes: one chunk, or for
+    ``full_prefill`` all 64 chunks of a 128K-token prompt (cache drawn once)."""
+    import workloads
+    if name == "full_prefill":
+        return [workloads.full_prefill_chunk(k) for k in range(64)]
+    return [workloads.by_name(name)]
+
+
+def run_ours(args, chunks):
     import torch
     import torch.distributed as dist
 
@@ -265,38 +287,61 @@ def run_ours(args, wl):
     torch.cuda.set_device(dev)
     ca.load_library()
 
-    mask_np = workloads.make_mask(wl)
-    Qh, Kh, Vh = workloads.make_qkv(wl)
-    mask = torch.from_numpy(mask_np).to(dev)
-    Q, K, V = Qh.to(dev), Kh.to(dev), Vh.to(dev)
-    tables = torch.empty((wl.B, wl.H_kv, wl.nKVmax), dtype=torch.int32, device=dev)
-    counts = torch.empty((wl.B, wl.H_kv), dtype=torch.int32, device=dev)
-    O = torch.empty_like(Q)
-    LSE = torch.empty((wl.B, wl.H_q, wl.C), dtype=torch.float32, device=dev)
-    ws = ca.new_workspace(wl.B, wl.H_q, wl.H_kv, wl.C, wl.blk, device=dev)
+    wl0 = chunks[-1]
+    Kh, Vh = workloads.make_kv(wl0)  # the cache every chunk of the step reads
+    K, V = Kh.to(dev), Vh.to(dev)
+    masks_np = [workloads.make_mask(w) for w in chunks]
+    Qs_h = [workloads.make_q(w) for w in chunks]
+    masks = [torch.from_numpy(m).to(dev) for m in masks_np]
+    Qs = [q.to(dev) for q in Qs_h]
+    tables = [torch.empty((w.B, w.H_kv, w.nKVmax), dtype=torch.int32, device=dev) for w in chunks]
+    counts = [torch.empty((w.B, w.H_kv), dtype=torch.int32, device=dev) for w in chunks]
+    Os = [torch.empty_like(q) for q in Qs]
+    LSEs = [torch.empty((w.B, w.H_q, w.C), dtype=torch.float32, device=dev) for w in chunks]
+    ws = ca.new_workspace(wl0.B, wl0.H_q, wl0.H_kv, wl0.C, wl0.blk, device=dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    n = len(chunks)
+
+    def build_k(k):
+        ca.build_block_tables(masks[k], chunks[k].group, tables=tables[k], counts=counts[k])
+
+    def attend_k(k):
+        ca.chunk_attention(Qs[k], K, V, tables[k], counts[k], chunks[k].chunk_start, O=Os[k],
+                           LSE=LSEs[k], workspace=ws)
+
+    def dense_k(k):
+        ca.dense_chunk_attention(Qs[k], K, V, chunks[k].chunk_start, chunks[k].blk, O=Os[k],
+                                 LSE=LSEs[k], workspace=ws)
 
     def build():
-        ca.build_block_tables(mask, wl.group, tables=tables, counts=counts)
+        for k in range(n):
+            build_k(k)
 
     def attend():
-        ca.chunk_attention(Q, K, V, tables, counts, wl.chunk_start, O=O, LSE=LSE, workspace=ws)
+        for k in range(n):
+            attend_k(k)
 
     def dense():
-        ca.dense_chunk_attention(Q, K, V, wl.chunk_start, wl.blk, O=O, LSE=LSE, workspace=ws)
+        for k in range(n):
+            dense_k(k)
+
+    def step():  # chunked prefill: each chunk's tables, then its attention
+        for k in range(n):
+            build_k(k)
+            attend_k(k)
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local])
         torch.cuda.synchronize(dev)
 
-    def timed(fn, n, warm):
+    def timed(fn, steps, warm):
         for _ in range(warm):
             fn()
         barrier()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(n)]
+              for _ in range(steps)]
         for a, b in ev:
             flush.zero_()
             a.record(stream)
@@ -305,19 +350,21 @@ def run_ours(args, wl):
         barrier()
         return [a.elapsed_time(b) for a, b in ev]
 
-    # work count of one step (from this step's own tables)
+    # work count of one step (from the step's own tables)
     build()
     torch.cuda.synchronize(dev)
-    T_np, c_np = tables.cpu().numpy(), counts.cpu().numpy()
-    pairs = visible_pairs(T_np, c_np, wl.chunk_start, wl.C, wl.blk, wl.group)
-    dense_pairs = visible_pairs(T_np, c_np, wl.chunk_start, wl.C, wl.blk, wl.group,
-                                dense_nkv=[-(-(cs + wl.C) // wl.blk) for cs in wl.chunk_start])
-    flops = 4.0 * wl.D * pairs
-    union = float(c_np.sum()) / float(sum(-(-(cs + wl.C) // wl.blk) for cs in wl.chunk_start) * wl.H_kv)
-
-    def step():
-        build()
-        attend()
+    flops = dense_flops = 0.0
+    union_num = union_den = 0
+    table_bytes = 0
+    for k, w in enumerate(chunks):
+        T_np, c_np = tables[k].cpu().numpy(), counts[k].cpu().numpy()
+        nkv = [-(-(cs + w.C) // w.blk) for cs in w.chunk_start]
+        flops += 4.0 * w.D * visible_pairs(T_np, c_np, w.chunk_start, w.C, w.blk, w.group)
+        dense_flops += 4.0 * w.D * visible_pairs(T_np, c_np, w.chunk_start, w.C, w.blk, w.group,
+                                                 dense_nkv=nkv)
+        union_num += int(c_np.sum())
+        union_den += sum(nkv) * w.H_kv
+        table_bytes += masks_np[k].nbytes + 4 * T_np.size + 4 * c_np.size
 
     gpu_index = local
     vis = os.environ.get("CUDA_VISIBLE_DEVICES")
@@ -334,36 +381,39 @@ def run_ours(args, wl):
     clocks = clk.summary()
     assert ca.read_device_status(ws) == ca.CA_OK, "device status not OK"
 
-    # end to end through the public API with pinned host buffers: per step the
-    # chunk's mask, queries and new K/V rows go up, O and LSE come back
-    cs0 = wl.chunk_start
-    mask_h = torch.from_numpy(mask_np).pin_memory()
-    Q_h = Qh.pin_memory()
-    Kc_h = torch.stack([Kh[b, :, cs0[b]:cs0[b] + wl.C] for b in range(wl.B)]).pin_memory()
-    Vc_h = torch.stack([Vh[b, :, cs0[b]:cs0[b] + wl.C] for b in range(wl.B)]).pin_memory()
-    O_h = torch.empty(O.shape, dtype=O.dtype).pin_memory()
-    LSE_h = torch.empty(LSE.shape, dtype=LSE.dtype).pin_memory()
+    # end to end through the public API with pinned host buffers: per chunk its
+    # mask, queries and new K/V rows go up, O and LSE come back
+    masks_h = [torch.from_numpy(m).pin_memory() for m in masks_np]
+    Qs_hp = [q.pin_memory() for q in Qs_h]
+    Kc_h, Vc_h = [], []
+    for w in chunks:
+        cs = w.chunk_start
+        Kc_h.append(torch.stack([Kh[b, :, cs[b]:cs[b] + w.C] for b in range(w.B)]).pin_memory())
+        Vc_h.append(torch.stack([Vh[b, :, cs[b]:cs[b] + w.C] for b in range(w.B)]).pin_memory())
+    Os_h = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in Os]
+    LSEs_h = [torch.empty(l.shape, dtype=l.dtype).pin_memory() for l in LSEs]
 
     def e2e_step():
-        mask.copy_(mask_h, non_blocking=True)
-        Q.copy_(Q_h, non_blocking=True)
-        for b in range(wl.B):
-            K[b, :, cs0[b]:cs0[b] + wl.C].copy_(Kc_h[b], non_blocking=True)
-            V[b, :, cs0[b]:cs0[b] + wl.C].copy_(Vc_h[b], non_blocking=True)
-        ca.build_block_tables(mask, wl.group, tables=tables, counts=counts)
-        ca.chunk_attention(Q, K, V, tables, counts, wl.chunk_start, O=O, LSE=LSE, workspace=ws)
-        O_h.copy_(O, non_blocking=True)
-        LSE_h.copy_(LSE, non_blocking=True)
+        for k, w in enumerate(chunks):
+            cs = w.chunk_start
+            masks[k].copy_(masks_h[k], non_blocking=True)
+            Qs[k].copy_(Qs_hp[k], non_blocking=True)
+            for b in range(w.B):
+                K[b, :, cs[b]:cs[b] + w.C].copy_(Kc_h[k][b], non_blocking=True)
+                V[b, :, cs[b]:cs[b] + w.C].copy_(Vc_h[k][b], non_blocking=True)
+            build_k(k)
+            attend_k(k)
+            Os_h[k].copy_(Os[k], non_blocking=True)
+            LSEs_h[k].copy_(LSEs[k], non_blocking=True)
 
     e2e_ms = timed(e2e_step, args.steps, args.warmup)
-    h2d = (mask_h.numel() + Q_h.numel() * 2 + Kc_h.numel() * 2 + Vc_h.numel() * 2)
-    d2h = O_h.numel() * 2 + LSE_h.numel() * 4
+    h2d = sum(m.numel() + 2 * q.numel() + 2 * kc.numel() + 2 * vc.numel()
+              for m, q, kc, vc in zip(masks_h, Qs_hp, Kc_h, Vc_h))
+    d2h = sum(2 * o.numel() + 4 * l.numel() for o, l in zip(Os_h, LSEs_h))
 
     def agg(ms_list):
         t = torch.tensor([sum(ms_list)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks(t, world)
 
     total_step = agg(step_ms)
     total_attn = agg(attn_ms)
@@ -373,40 +423,42 @@ def run_ours(args, wl):
     K_ = args.steps
     value = world * K_ * flops / (total_step * 1e-3) / 1e12
     attn_tflops = flops / (total_attn / K_ * 1e-3) / 1e12
-    dense_flops = 4.0 * wl.D * dense_pairs
     peaks, peak_kind = _peaks()
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     peak_sus = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    name = "full_prefill" if n > 1 else wl0.name
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": K_, "warmup": args.warmup, "ms_per_step": total_step / K_,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic", "config": _config(wl),
+        "data": "synthetic", "config": _config(wl0, name, n),
         "attn_ms": total_attn / K_, "attn_tflops": attn_tflops,
         "build_us": total_build / K_ * 1e3,
-        "build_gbs": (mask_np.nbytes + 4 * T_np.size + 4 * c_np.size) / (total_build / K_ * 1e-3) / 1e9,
+        "build_gbs": table_bytes / (total_build / K_ * 1e-3) / 1e9,
         "dense_ms": total_dense / K_,
         "dense_tflops": dense_flops / (total_dense / K_ * 1e-3) / 1e12,
         "speedup_vs_dense": total_dense / total_step,
-        "union_density": union,
+        "union_density": union_num / union_den,
         "effective_tflop_per_step": flops / 1e12,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": attn_tflops / peak,
-                     "traffic": profiled_traffic(wl.name),
+                     "traffic": profiled_traffic(name) if n == 1 else None,
                      "peak_source": f"{peak_kind} bf16 burst (kernel timed alone, L2 flushed)",
                      "frac_of_sustained_peak": attn_tflops / peak_sus,
-                     "algorithmic_flop_per_launch": flops,
+                     "algorithmic_flop_per_launch": flops / n,
                      "kernel": "chunk_attn_kernel"},
         "e2e": {"value": world * K_ * flops / (total_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
-        "gpu_launches": 2 * K_,
+        "gpu_launches": 2 * n * K_,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, n, dt, threads = oracle_sample_rate(wl, mask_np, Qh, Kh, Vh, target_s=args.cpu_seconds)
+        last = chunks[-1]
+        v, nrows, dt, threads = oracle_sample_rate(last, masks_np[-1], Qs_h[-1], Kh, Vh,
+                                                   target_s=args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                                "sample": f"{n} seeded query rows of {wl.B * wl.H_q * wl.C} "
-                                          f"({dt:.1f} s, fp64)"}
+                                "sample": f"{nrows} seeded query rows of {last.B * last.H_q * last.C}"
+                                          f" of chunk {last.name} ({dt:.1f} s, fp64)"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -427,11 +479,10 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    import workloads
-    wl = workloads.by_name(args.workload)
+    chunks = step_chunks(args.workload)
     if args.impl == "reference":
-        return run_reference(args, wl)
-    return run_ours(args, wl)
+        return run_reference(args, chunks[-1], args.workload)
+    return run_ours(args, chunks)
 
 
 if __name__ == "__main__":

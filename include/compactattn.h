@@ -157,6 +157,13 @@ int ca_chunk_attention_noalloc(const void *Q, const void *K, const void *V, cons
                                int H_kv, int C, int L_max, int D, int blk, float scale, void *O,
                                float *LSE, unsigned int *device_status, void *stream);
 
+/* Self-test of the kernels' bounded waits: one kernel waits on a barrier that
+ * nothing ever completes; after limit_cycles SM clock cycles (at most about
+ * 2 s) the wait gives up, sets the timeout bit of the workspace status word
+ * and the kernel returns. ca_read_device_status() then reports CA_ERR_TIMEOUT
+ * and the context stays usable. Nothing faults, traps or hangs. */
+int ca_selftest_bounded_wait(void *workspace, long long limit_cycles, void *stream);
+
 /* Synchronises `stream`, then reads the workspace status word written by the
  * kernels: CA_OK, CA_ERR_TABLE or CA_ERR_TIMEOUT (sticky until the workspace is
  * zeroed again; CA_ERR_TABLE wins if both are set). CA_ERR_CUDA if the stream

@@ -64,6 +64,7 @@ EXPORTED_SYMBOLS = (
     "ca_dense_chunk_attention",
     "ca_read_device_status",
     "ca_chunk_attention_noalloc",
+    "ca_selftest_bounded_wait",
 )
 
 
@@ -105,6 +106,8 @@ def load_library():
         lib.ca_chunk_attention_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P, P,
                                                    P, P]
         lib.ca_chunk_attention_noalloc.restype = I
+        lib.ca_selftest_bounded_wait.argtypes = [P, ctypes.c_longlong, P]
+        lib.ca_selftest_bounded_wait.restype = I
         _lib = lib
         return lib
 
@@ -274,6 +277,15 @@ def dense_chunk_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
                                       workspace.numel(), _stream_handle(stream, Q.device))
     _check("ca_dense_chunk_attention", st)
     return O, LSE
+
+
+def selftest_bounded_wait(workspace: torch.Tensor, limit_cycles: int = 20_000_000,
+                          stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Runs the bounded-wait self-test kernel (a wait that nothing completes
+    gives up after ``limit_cycles`` and records a timeout in ``workspace``)."""
+    st = load_library().ca_selftest_bounded_wait(_ptr(workspace), int(limit_cycles),
+                                                 _stream_handle(stream, workspace.device))
+    _check("ca_selftest_bounded_wait", st)
 
 
 def read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:

@@ -94,14 +94,15 @@ struct AbortState {
 // Waits until the phase with the given parity of `bar` has completed.
 // Returns false (and records kDevErrTimeout) if the wait exceeded the limit or
 // the CTA is aborting.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const AbortState &ab) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const AbortState &ab,
+                                          long long limit_cycles = kWaitLimitCycles) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(a, parity)) return true;
         if (*ab.flag) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit_cycles) {
             *ab.flag = 1;
             atomicOr(ab.status, kDevErrTimeout);
             return false;
