@@ -132,6 +132,35 @@ int ca_dense_chunk_attention(const void *Q, const void *K, const void *V,
                              void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Explicit-compaction ablation, step 1 (pages: "Experimental results" — the
+ * efficiency ablation comparing zero-copy paged execution with explicit KV
+ * compaction, the copy that token-level selection methods need): gathers the
+ * K and V blocks each table selects into compact buffers. Block
+ * tables[b,g,t] (t < counts[b,g]) of K / V is copied to rows
+ * [t*blk, (t+1)*blk) of Kc / Vc; entries outside [0, nKVmax) give zero rows;
+ * rows at t >= counts[b,g] are not written.
+ * K, V, Kc, Vc bf16 [B, H_kv, L_max, D] (16-byte aligned); tables / counts as
+ * for ca_chunk_attention. Errors: CA_ERR_INVALID_ARG, CA_ERR_SHAPE,
+ * CA_ERR_ALIGN, CA_ERR_UNSUPPORTED, CA_ERR_CUDA.
+ */
+int ca_compact_kv_blocks(const void *K, const void *V, const int32_t *tables,
+                         const int32_t *counts, int B, int H_kv, int L_max, int D, int blk,
+                         void *Kc, void *Vc, void *stream);
+
+/*
+ * Explicit-compaction ablation, step 2: ca_chunk_attention over the compact
+ * buffers of ca_compact_kv_blocks — block t of a table is read from rows
+ * [t*blk, (t+1)*blk) of Kc / Vc and masked by its original position
+ * tables[b,g,t]*blk. Same arguments, results and errors as
+ * ca_chunk_attention, with Kc / Vc in place of K / V.
+ */
+int ca_compacted_chunk_attention(const void *Q, const void *Kc, const void *Vc,
+                                 const int32_t *tables, const int32_t *counts,
+                                 const int32_t *chunk_start, int B, int H_q, int H_kv, int C,
+                                 int L_max, int D, int blk, float scale, void *O, float *LSE,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * ca_chunk_attention without a caller workspace, for callers that cannot
  * allocate device memory when they run attention (an engine whose device
  * memory is sized once at start-up, code inside a fixed memory pool, a host

@@ -36,6 +36,8 @@ __all__ = [
     "dense_chunk_attention",
     "read_device_status",
     "chunk_attention_noalloc",
+    "compact_kv_blocks",
+    "compacted_chunk_attention",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -65,6 +67,8 @@ EXPORTED_SYMBOLS = (
     "ca_read_device_status",
     "ca_chunk_attention_noalloc",
     "ca_selftest_bounded_wait",
+    "ca_compact_kv_blocks",
+    "ca_compacted_chunk_attention",
 )
 
 
@@ -108,6 +112,11 @@ def load_library():
         lib.ca_chunk_attention_noalloc.restype = I
         lib.ca_selftest_bounded_wait.argtypes = [P, ctypes.c_longlong, P]
         lib.ca_selftest_bounded_wait.restype = I
+        lib.ca_compact_kv_blocks.argtypes = [P, P, P, P, I, I, I, I, I, P, P, P]
+        lib.ca_compact_kv_blocks.restype = I
+        lib.ca_compacted_chunk_attention.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P,
+                                                     P, P, S, P]
+        lib.ca_compacted_chunk_attention.restype = I
         _lib = lib
         return lib
 
@@ -334,4 +343,62 @@ def chunk_attention_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
         L_max // nK, float(scale), _ptr(O), _ptr(LSE), _ptr(device_status),
         _stream_handle(stream, Q.device))
     _check("ca_chunk_attention_noalloc", st)
+    return O, LSE
+
+
+# ----------------------------------------------------------------- ablation
+
+def compact_kv_blocks(K: torch.Tensor, V: torch.Tensor, tables: torch.Tensor,
+                      counts: torch.Tensor, Kc: Optional[torch.Tensor] = None,
+                      Vc: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None
+                      ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Explicit-compaction ablation: gathers the blocks each table selects into
+    compact K / V buffers (block t of table (b, g) at rows [t*blk, (t+1)*blk))."""
+    _need(K, "K", torch.bfloat16, 4)
+    _need(V, "V", torch.bfloat16, 4)
+    _need(tables, "tables", torch.int32, 3)
+    _need(counts, "counts", torch.int32, 2)
+    B, H_kv, L_max, D = K.shape
+    nK = tables.shape[-1]
+    if nK <= 0 or L_max % nK:
+        raise ValueError("tables' last dim must divide L_max (it is L_max / blk)")
+    if Kc is None:
+        Kc = torch.zeros_like(K)
+    if Vc is None:
+        Vc = torch.zeros_like(V)
+    _need(Kc, "Kc", torch.bfloat16, 4)
+    _need(Vc, "Vc", torch.bfloat16, 4)
+    st = load_library().ca_compact_kv_blocks(_ptr(K), _ptr(V), _ptr(tables), _ptr(counts), B,
+                                             H_kv, L_max, D, L_max // nK, _ptr(Kc), _ptr(Vc),
+                                             _stream_handle(stream, K.device))
+    _check("ca_compact_kv_blocks", st)
+    return Kc, Vc
+
+
+def compacted_chunk_attention(Q: torch.Tensor, Kc: torch.Tensor, Vc: torch.Tensor,
+                              tables: torch.Tensor, counts: torch.Tensor,
+                              chunk_start: Sequence[int], scale: Optional[float] = None,
+                              O: Optional[torch.Tensor] = None, LSE: Optional[torch.Tensor] = None,
+                              workspace: Optional[torch.Tensor] = None,
+                              stream: Optional[torch.cuda.Stream] = None
+                              ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Explicit-compaction ablation: chunk_attention over compact_kv_blocks'
+    buffers (same results as chunk_attention on the original cache)."""
+    _need(tables, "tables", torch.int32, 3)
+    _need(counts, "counts", torch.int32, 2)
+    nK = tables.shape[-1]
+    L_max = Kc.shape[2]
+    if nK <= 0 or L_max % nK:
+        raise ValueError("tables' last dim must divide L_max (it is L_max / blk)")
+    blk = L_max // nK
+    B, H_q, H_kv, C, L_max, D, O, LSE, workspace = _attn_common(Q, Kc, Vc, O, LSE, workspace, blk)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    cs = _chunk_start_host(chunk_start, B)
+    st = load_library().ca_compacted_chunk_attention(
+        _ptr(Q), _ptr(Kc), _ptr(Vc), _ptr(tables), _ptr(counts), cs, B, H_q, H_kv, C, L_max, D,
+        blk, float(scale), _ptr(O), _ptr(LSE), _ptr(workspace), workspace.numel(),
+        _stream_handle(stream, Q.device))
+    _check("ca_compacted_chunk_attention", st)
     return O, LSE

@@ -31,6 +31,20 @@ struct AttnArgs {
     void *workspace;
 };
 
-int launch_chunk_attention(const AttnArgs &a, bool dense, cudaStream_t stream);
+// Attention kernel modes: walk the tables over the cache in place; every block
+// of the visible length (the dense path); or the tables' blocks gathered into a
+// compact buffer (block t of a table at row t * blk, masked by its original
+// position — the explicit-compaction ablation).
+constexpr int kModeTables = 0;
+constexpr int kModeDense = 1;
+constexpr int kModeCompact = 2;
+
+int launch_chunk_attention(const AttnArgs &a, int mode, cudaStream_t stream);
+
+// Copies the K and V blocks each table selects into compact buffers: block
+// tables[b,g,t] of the cache goes to rows [t * blk, (t + 1) * blk) of Kc / Vc.
+int launch_compact_kv(const void *K, const void *V, const int32_t *tables, const int32_t *counts,
+                      int B, int H_kv, int L_max, int D, int blk, void *Kc, void *Vc,
+                      cudaStream_t stream);
 
 }  // namespace ca

@@ -98,7 +98,7 @@ int ca_chunk_attention(const void *Q, const void *K, const void *V, const int32_
     if (st != CA_OK) return st;
     ca::AttnArgs a{Q, K, V, tables, counts, chunk_start, B, H_q, H_kv, C, L_max, D, blk,
                    scale, O, LSE, workspace};
-    return ca::launch_chunk_attention(a, false, static_cast<cudaStream_t>(stream));
+    return ca::launch_chunk_attention(a, ca::kModeTables, static_cast<cudaStream_t>(stream));
 }
 
 int ca_dense_chunk_attention(const void *Q, const void *K, const void *V,
@@ -110,7 +110,35 @@ int ca_dense_chunk_attention(const void *Q, const void *K, const void *V,
     if (st != CA_OK) return st;
     ca::AttnArgs a{Q, K, V, nullptr, nullptr, chunk_start, B, H_q, H_kv, C, L_max, D, blk,
                    scale, O, LSE, workspace};
-    return ca::launch_chunk_attention(a, true, static_cast<cudaStream_t>(stream));
+    return ca::launch_chunk_attention(a, ca::kModeDense, static_cast<cudaStream_t>(stream));
+}
+
+int ca_compact_kv_blocks(const void *K, const void *V, const int32_t *tables,
+                         const int32_t *counts, int B, int H_kv, int L_max, int D, int blk,
+                         void *Kc, void *Vc, void *stream) {
+    if (!K || !V || !tables || !counts || !Kc || !Vc) return CA_ERR_INVALID_ARG;
+    if (B <= 0 || H_kv <= 0 || L_max <= 0 || D <= 0 || blk <= 0) return CA_ERR_INVALID_ARG;
+    if (L_max % blk != 0) return CA_ERR_SHAPE;
+    if (!(D == 64 || D == 128) || !(blk == 64 || blk == 128)) return CA_ERR_UNSUPPORTED;
+    if ((long long)B * H_kv * L_max >= (1LL << 31)) return CA_ERR_SHAPE;
+    if (!aligned(K, 16) || !aligned(V, 16) || !aligned(Kc, 16) || !aligned(Vc, 16) ||
+        !aligned(tables, 4) || !aligned(counts, 4))
+        return CA_ERR_ALIGN;
+    return ca::launch_compact_kv(K, V, tables, counts, B, H_kv, L_max, D, blk, Kc, Vc,
+                                 static_cast<cudaStream_t>(stream));
+}
+
+int ca_compacted_chunk_attention(const void *Q, const void *Kc, const void *Vc,
+                                 const int32_t *tables, const int32_t *counts,
+                                 const int32_t *chunk_start, int B, int H_q, int H_kv, int C,
+                                 int L_max, int D, int blk, float scale, void *O, float *LSE,
+                                 void *workspace, size_t workspace_bytes, void *stream) {
+    const int st = check_attention(Q, Kc, Vc, tables, counts, false, chunk_start, B, H_q, H_kv,
+                                   C, L_max, D, blk, scale, O, LSE, workspace, workspace_bytes);
+    if (st != CA_OK) return st;
+    ca::AttnArgs a{Q, Kc, Vc, tables, counts, chunk_start, B, H_q, H_kv, C, L_max, D, blk,
+                   scale, O, LSE, workspace};
+    return ca::launch_chunk_attention(a, ca::kModeCompact, static_cast<cudaStream_t>(stream));
 }
 
 int ca_read_device_status(const void *workspace, void *stream) {

@@ -165,12 +165,14 @@ __device__ __forceinline__ void tmem_ld_row<64>(uint32_t taddr, uint32_t (&r)[64
     tmem_ld64(taddr, r);
 }
 
-template <int D, int BLK, bool DENSE>
+template <int D, int BLK, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params P) {
     using L = Layout<D, BLK>;
+    constexpr bool DENSE = MODE == kModeDense;
+    constexpr bool COMPACT = MODE == kModeCompact;  // K/V block t sits at row t * BLK
     constexpr int NST = L::kStages;
     constexpr int DCH = D / 64;  // 64-element (128-byte) sub-tiles along D
     constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, BLK, false);
@@ -297,8 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (out) jb = P.nKVmax;
                 }
                 for (int q = 0; q < nwin; ++q) {
-                    const int blk_idx = __shfl_sync(0xffffffffu, jb, q);
                     const int j = w0 + q;
+                    const int blk_idx = COMPACT ? j : __shfl_sync(0xffffffffu, jb, q);
                     const int s = j % NST;
                     const uint32_t ph = ((j / NST) & 1) ^ 1;
                     int good = 1;
@@ -608,10 +610,10 @@ bool encode_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uin
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int BLK, bool DENSE>
+template <int D, int BLK, int MODE>
 int launch_t(const AttnArgs &a, cudaStream_t stream) {
     using L = Layout<D, BLK>;
-    auto kern = chunk_attn_kernel<D, BLK, DENSE>;
+    auto kern = chunk_attn_kernel<D, BLK, MODE>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -680,10 +682,13 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
 
 }  // namespace
 
-int launch_chunk_attention(const AttnArgs &a, bool dense, cudaStream_t stream) {
-#define CA_DISPATCH(D_, BLK_)                                                    \
-    if (a.D == D_ && a.blk == BLK_)                                              \
-        return dense ? launch_t<D_, BLK_, true>(a, stream) : launch_t<D_, BLK_, false>(a, stream);
+int launch_chunk_attention(const AttnArgs &a, int mode, cudaStream_t stream) {
+#define CA_DISPATCH(D_, BLK_)                                                         \
+    if (a.D == D_ && a.blk == BLK_) {                                                 \
+        if (mode == kModeDense) return launch_t<D_, BLK_, kModeDense>(a, stream);     \
+        if (mode == kModeCompact) return launch_t<D_, BLK_, kModeCompact>(a, stream); \
+        return launch_t<D_, BLK_, kModeTables>(a, stream);                            \
+    }
     CA_DISPATCH(128, 128)
     CA_DISPATCH(128, 64)
     CA_DISPATCH(64, 128)
