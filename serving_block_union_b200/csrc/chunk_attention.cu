@@ -66,17 +66,29 @@ constexpr int kTileM = 128;
 #ifndef CA_REG_SPLIT
 #define CA_REG_SPLIT 1
 #endif
+// Softmax warps per row: 1 (a thread owns a whole S row) or 2 (two warps on the
+// same TMEM lanes take one half of the row's columns each, and exchange their
+// partial row maxima and sums through shared memory).
+#ifndef CA_COL_SPLIT
+#define CA_COL_SPLIT 1
+#endif
+constexpr int kColSplit = CA_COL_SPLIT;
+static_assert(kColSplit == 1 || kColSplit == 2, "column split must be 1 or 2");
 constexpr bool kRegSplit = CA_REG_SPLIT != 0;
-constexpr int kThreads = kRegSplit ? 384 : 320;
-constexpr int kMmaWarp = 8;
-constexpr int kTmaWarp = 9;
-constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxWarps = 8 * kColSplit;
+constexpr int kMmaWarp = kSoftmaxWarps;
+constexpr int kTmaWarp = kSoftmaxWarps + 1;
+// control warpgroup padded to 4 warps when the register split needs whole warpgroups
+constexpr int kThreads = 32 * (kSoftmaxWarps + (kRegSplit ? 4 : 2));
+constexpr int kLaunchRegs = kColSplit == 1 ? 168 : 96;
 #ifndef CA_SOFTMAX_REGS
-#define CA_SOFTMAX_REGS 208
+#define CA_SOFTMAX_REGS (CA_COL_SPLIT == 1 ? 208 : 104)
 #endif
 constexpr int kSoftmaxRegs = CA_SOFTMAX_REGS;
-constexpr int kControlRegs = 3 * kLaunchRegs - 2 * kSoftmaxRegs;
-static_assert(2 * kSoftmaxRegs + kControlRegs == 3 * kLaunchRegs, "register split must balance");
+// per SM sub-partition: one warp of each softmax warpgroup plus one control warp
+constexpr int kControlRegs = (2 * kColSplit + 1) * kLaunchRegs - 2 * kColSplit * kSoftmaxRegs;
+static_assert(2 * kColSplit * kSoftmaxRegs + kControlRegs == (2 * kColSplit + 1) * kLaunchRegs,
+              "register split must balance");
 static_assert(kSoftmaxRegs % 8 == 0 && kControlRegs % 8 == 0 && kControlRegs >= 24,
               "setmaxnreg counts are multiples of 8, at least 24");
 constexpr uint32_t kTmemCols = 512;
@@ -115,10 +127,12 @@ struct Layout {
     static constexpr int kKOff = 2 * kQTile;
     static constexpr int kVOff = kKOff + kStages * kKV;
     static constexpr int kBarOff = kVOff + kStages * kKV;
-    static constexpr int kPChunkKeys = kPChunkKeysCfg < BLK ? kPChunkKeysCfg : BLK;
+    static constexpr int kPChunkKeys =
+        kColSplit == 2 ? BLK / 2 : (kPChunkKeysCfg < BLK ? kPChunkKeysCfg : BLK);
     static constexpr int kPChunks = BLK / kPChunkKeys;  // P reaches the MMA chunk by chunk
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 * kPChunks + 2 + 1;
-    static constexpr int kEnd = kBarOff + kNumBars * 8 + 16;
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 * kPChunks + 2 + 1 + 8;
+    static constexpr int kXchOff = kBarOff + kNumBars * 8 + 16;  // [2][4][2][32] floats
+    static constexpr int kEnd = kXchOff + 2 * 4 * 2 * 32 * 4;
     static constexpr int kDynamic = (kEnd + 1024) > kSmemFloor ? (kEnd + 1024) : kSmemFloor;
     static_assert(kStages >= 2, "need at least two K/V stages");
     static_assert(kDynamic <= kSmemBudget, "shared memory budget exceeded");
@@ -164,6 +178,10 @@ template <>
 __device__ __forceinline__ void tmem_ld_row<64>(uint32_t taddr, uint32_t (&r)[64]) {
     tmem_ld64(taddr, r);
 }
+template <>
+__device__ __forceinline__ void tmem_ld_row<32>(uint32_t taddr, uint32_t (&r)[32]) {
+    tmem_ld32(taddr, r);
+}
 
 template <int D, int BLK, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -194,7 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *p_full = s_full + 2;      // [2][NPC]: P chunk c of tile t stored in TMEM
     uint64_t *o_full = p_full + 2 * NPC;  // [2]
     uint64_t *mma_done = o_full + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    uint64_t *xch_bar = mma_done + 1;  // [2 tiles][4 quarters]: the two half-row warps meet
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xch_bar + 8);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -229,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(o_full + t, 1);
         }
         mbar_init(mma_done, 1);
+        for (int x = 0; x < 8; ++x) mbar_init(xch_bar + x, 2);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -427,7 +447,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         if (kRegSplit) regs_inc<kSoftmaxRegs>();
         // ================================================================ softmax
-        const int t = warp >> 2;
+        // Warp (t, hf, qw): tile t, column part hf of the S row (kColSplit parts),
+        // TMEM lanes / packed rows 32*qw .. 32*qw + 31.
+        constexpr int CW = BLK / kColSplit;   // S columns (keys) per warp
+        constexpr int DW = D / kColSplit;     // O columns per warp
+        constexpr int CPW = NPC / kColSplit;  // P chunks per warp
+        const int t = warp / (4 * kColSplit);
+        const int hf = (warp / 4) % kColSplit;
         const int qw = warp & 3;
         const int m = qw * 32 + lane;
         const int h_local = m / R;
@@ -437,10 +463,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h = g * P.G + h_local;
         const uint32_t lane_base = static_cast<uint32_t>(qw * 32) << 16;
         const uint32_t tS = tmem + lane_base + t * 128;
-        const uint32_t tO = tmem + lane_base + 256 + t * 128;
+        const uint32_t tO = tmem + lane_base + 256 + t * 128 + hf * DW;
         const float sl2 = P.scale_log2;
+        // partner exchange (column split only): partial row max / sum of the
+        // other half, through shared memory and a bounded mbarrier
+        float *xch = reinterpret_cast<float *>(smem + L::kXchOff);
+        float *xch_mine = xch + ((t * 4 + qw) * 2 + hf) * 32 + lane;
+        const float *xch_other = xch + ((t * 4 + qw) * 2 + (1 - hf)) * 32 + lane;
+        uint64_t *xbar = xch_bar + t * 4 + qw;
+        uint32_t xph = 0;
+        auto exchange = [&](float mine, float &other) -> bool {
+            *xch_mine = mine;
+            __syncwarp();
+            mbar_arrive_lane0(xbar, lane);
+            const bool got = mbar_wait(xbar, xph & 1, ab);
+            ++xph;
+            if (!__all_sync(0xffffffffu, got)) return false;
+            other = *xch_other;
+            return true;
+        };
 
-        float m_run = -INFINITY, l_run = 0.0f;
+        float m_run = -INFINITY, l_run = 0.0f;  // l_run: this warp's columns only
         bool ok = true;
         for (int j = 0; j < n_eff; ++j) {
             ok = mbar_wait(s_full + t, j & 1, ab);
@@ -449,19 +492,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            float s[BLK];
+            float s[CW];
             {
-                uint32_t v[BLK];
-                tmem_ld_row<BLK>(tS, v);  // the whole S row in one TMEM round trip
+                uint32_t v[CW];
+                tmem_ld_row<CW>(tS + hf * CW, v);  // this warp's S columns in one round trip
 #pragma unroll
-                for (int i = 0; i < BLK; ++i) s[i] = __uint_as_float(v[i]);
+                for (int i = 0; i < CW; ++i) s[i] = __uint_as_float(v[i]);
             }
             if (j >= n_full) {
                 int jb = DENSE ? j : __ldg(T + j);
                 jb = min(max(jb, 0), P.nKVmax);  // only matters for a flagged, invalid table
-                const int lim = p - jb * BLK;    // keys jb*BLK + c with c <= lim are visible
+                const int lim = p - jb * BLK - hf * CW;  // columns c <= lim are visible
 #pragma unroll
-                for (int c = 0; c < BLK; ++c)
+                for (int c = 0; c < CW; ++c)
                     if (c > lim) s[c] = -INFINITY;
             }
             // row max: 8 independent chains of 3-input max, then a short tree
@@ -469,15 +512,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 8; ++k) mx8[k] = s[k];
 #pragma unroll
-            for (int c = 8; c + 8 < BLK; c += 16)
+            for (int c = 8; c + 8 < CW; c += 16)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], s[c + k], s[c + 8 + k]);
-            if ((BLK - 8) % 16 != 0) {
+            if ((CW - 8) % 16 != 0) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], s[BLK - 8 + k]);
+                for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], s[CW - 8 + k]);
             }
-            const float m_blk = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
-                                      fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7])) * sl2;
+            float pmax = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
+                               fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
+            if (kColSplit == 2) {
+                float other;
+                if (!exchange(pmax, other)) {
+                    ok = false;
+                    break;
+                }
+                pmax = fmaxf(pmax, other);
+            }
+            const float m_blk = pmax * sl2;
             const float m_new = fmaxf(m_run, m_blk);
             const bool old_finite = m_run != -INFINITY;
             const bool upd = old_finite ? (m_new > m_run + kRescaleThreshold)
@@ -489,12 +541,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // O rescale (rare: only when a row's max grew past the threshold). O is
             // stable here: S(j) was committed after P.V(j-1) was issued. It must land
-            // before the first P chunk is handed over.
+            // before the first P chunk is handed over. Each warp rescales its
+            // DW columns of O.
             const bool need = upd && old_finite && j > 0;
             if (__any_sync(0xffffffffu, need)) {
                 const float a = need ? alpha : 1.0f;
 #pragma unroll
-                for (int c = 0; c < D / 16; ++c) {
+                for (int c = 0; c < DW / 16; ++c) {
                     uint32_t v[16];
                     tmem_ld16(tO + c * 16, v);
 #pragma unroll
@@ -513,14 +566,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc2[k] = 0ull;
 #pragma unroll
-            for (int c = 0; c < NPC; ++c) {
+            for (int cl = 0; cl < CPW; ++cl) {
                 constexpr int CK = L::kPChunkKeys;
+                const int c = hf * CPW + cl;  // P chunk index within the row
                 uint32_t pk[CK / 2];
 #pragma unroll
                 for (int i = 0; i < CK / 2; ++i) {
-                    const int e0 = c * CK + 2 * i;
+                    const int e0 = cl * CK + 2 * i;  // element in this warp's s[]
                     const uint64_t x2 = f2_fma(f2_pack(s[e0], s[e0 + 1]), sl2x2, nm2);
-                    const uint64_t p2 = use_poly_pair(e0 / 2)
+                    const uint64_t p2 = use_poly_pair(c * CK / 2 + i)
                                             ? exp2_poly2(x2)
                                             : f2_pack(ex2_approx(f2_lo(x2)), ex2_approx(f2_hi(x2)));
                     acc2[i & 3] = f2_add(acc2[i & 3], p2);
@@ -543,10 +597,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             have_o = __all_sync(0xffffffffu, got);
             tc_fence_after();
         }
+        if (kColSplit == 2 && have_o) {
+            float other = 0.0f;
+            if (exchange(l_run, other)) {
+                l_run += other;
+            } else {
+                have_o = false;
+            }
+        }
         const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-        uint16_t *orow = P.O + (((size_t)b * P.H_q + h) * P.C + r) * D;
+        uint16_t *orow = P.O + (((size_t)b * P.H_q + h) * P.C + r) * D + hf * DW;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < DW / 32; ++c) {
             uint32_t v[32];
             if (have_o) {
                 tmem_ld32(tO + c * 32, v);
@@ -566,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
             }
         }
-        if (valid && P.LSE != nullptr) {
+        if (valid && hf == 0 && P.LSE != nullptr) {
             P.LSE[((size_t)b * P.H_q + h) * P.C + r] =
                 (l_run > 0.0f && have_o) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
         }
