@@ -245,13 +245,25 @@ int oracle_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *
         J->end = n_rows * (w + 1) / n_threads;
         J->status = ORACLE_OK;
     }
-    for (int w = 1; w < n_threads; ++w) pthread_create(&tid[w], NULL, attn_worker, &jobs[w]);
+    /* A job whose thread cannot be started runs on this thread instead, so
+     * every row is computed whatever the process's thread limit. */
+    char *started = (char *)calloc((size_t)n_threads, 1);
+    if (!started) {
+        free(jobs);
+        free(tid);
+        return ORACLE_ENOMEM;
+    }
+    for (int w = 1; w < n_threads; ++w)
+        started[w] = pthread_create(&tid[w], NULL, attn_worker, &jobs[w]) == 0;
     attn_worker(&jobs[0]);
+    for (int w = 1; w < n_threads; ++w)
+        if (!started[w]) attn_worker(&jobs[w]);
     int status = jobs[0].status;
     for (int w = 1; w < n_threads; ++w) {
-        pthread_join(tid[w], NULL);
+        if (started[w]) pthread_join(tid[w], NULL);
         if (jobs[w].status != ORACLE_OK) status = jobs[w].status;
     }
+    free(started);
     free(jobs);
     free(tid);
     return status;
