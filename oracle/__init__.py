@@ -49,6 +49,12 @@ def _load():
             lib.oracle_attention_rows.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I,
                                                   ctypes.c_double, P, ctypes.c_int64, P, P, I]
             lib.oracle_attention_rows.restype = I
+            lib.oracle_attention_tile_rows.argtypes = [P, P, P, P, I, P, I, I, I, I, I, I, I,
+                                                       ctypes.c_double, P, ctypes.c_int64, P, P,
+                                                       I]
+            lib.oracle_attention_tile_rows.restype = I
+            lib.oracle_tile_span_tables.argtypes = [P, I, I, I, I, I, P, P]
+            lib.oracle_tile_span_tables.restype = I
             lib.oracle_visible_pairs.argtypes = [P, P, P, I, I, I, I, I, I]
             lib.oracle_visible_pairs.restype = ctypes.c_int64
             _lib = lib
@@ -131,6 +137,62 @@ def attention(Q, K, V, chunk_start: Sequence[int], blk: int, tables=None, counts
     if rows is None:
         return O.reshape(B, H_q, C, D), LSE.reshape(B, H_q, C)
     return O, LSE
+
+
+def attention_tile(Q, K, V, chunk_start: Sequence[int], blk: int, mask,
+                   scale: Optional[float] = None, rows: Optional[np.ndarray] = None,
+                   threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """fp64 per-tile block-sparse chunk attention: row r of head h attends to
+    the keys k <= chunk_start[b] + r of the blocks its own Q-block selects,
+    ``mask[b, h, r // blk, k // blk] != 0`` (no Q-block or head union).
+
+    ``mask`` uint8 [B, H_q, nQ, L_max/blk]; the rest as in :func:`attention`."""
+    B, H_q, C, D = Q.shape
+    Bk, H_kv, L_max, Dk = K.shape
+    if Bk != B or Dk != D or tuple(V.shape) != tuple(K.shape):
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(D))
+    m = np.ascontiguousarray(mask, dtype=np.uint8)
+    if m.ndim != 4 or m.shape[:2] != (B, H_q) or m.shape[3] != L_max // blk:
+        raise ValueError("mask must be [B, H_q, nQ, L_max/blk]")
+    q, k, v = _bf16_bits(Q), _bf16_bits(K), _bf16_bits(V)
+    cs = np.ascontiguousarray(chunk_start, dtype=np.int32)
+    if cs.shape != (B,):
+        raise ValueError("chunk_start must have B entries")
+    r = None
+    n = B * H_q * C
+    if rows is not None:
+        r = np.ascontiguousarray(rows, dtype=np.int64)
+        n = r.size
+    O = np.empty((n, D), np.float64)
+    LSE = np.empty(n, np.float64)
+    st = _load().oracle_attention_tile_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(m), m.shape[2],
+                                            _ptr(cs), B, H_q, H_kv, C, L_max, D, blk,
+                                            float(scale), _ptr(r), n, _ptr(O), _ptr(LSE),
+                                            int(threads))
+    if st != 0:
+        raise ValueError(f"oracle_attention_tile_rows failed ({st})")
+    if rows is None:
+        return O.reshape(B, H_q, C, D), LSE.reshape(B, H_q, C)
+    return O, LSE
+
+
+def tile_span_tables(mask, span: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Span tables of the per-tile path: per (b, h, span of ``span`` Q-blocks)
+    the ascending KV blocks any Q-block of the span selects, each entry
+    ``j | bits << 24`` with bit u set iff Q-block ``span*s + u`` selects j;
+    padded with -1. Returns tables int32 [B, H_q, nS, nKVmax], counts int32
+    [B, H_q, nS], nS = ceil(nQ / span)."""
+    m = np.ascontiguousarray(mask, dtype=np.uint8)
+    B, H_q, nQ, nKVmax = m.shape
+    nS = -(-nQ // span)
+    T = np.empty((B, H_q, nS, nKVmax), np.int32)
+    c = np.empty((B, H_q, nS), np.int32)
+    st = _load().oracle_tile_span_tables(_ptr(m), B, H_q, nQ, nKVmax, span, _ptr(T), _ptr(c))
+    if st != 0:
+        raise ValueError(f"oracle_tile_span_tables failed ({st})")
+    return T, c
 
 
 def visible_pairs(chunk_start: Sequence[int], B: int, H_q: int, H_kv: int, C: int, L_max: int,

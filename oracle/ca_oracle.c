@@ -102,6 +102,8 @@ int oracle_block_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax,
 typedef struct {
     const uint16_t *Q, *K, *V;       /* bf16 bits */
     const int32_t *tables, *counts;  /* NULL tables: dense, T = [0, nKV_b) */
+    const uint8_t *tile_mask;        /* non-NULL: per-tile block-sparse key sets */
+    int nQ;                          /* Q-blocks per chunk (tile_mask only) */
     const int32_t *chunk_start;
     int B, H_q, H_kv, C, L_max, D, blk;
     double scale;
@@ -112,6 +114,10 @@ typedef struct {
     int status;
 } attn_job;
 
+static int attention_over_keys(const attn_job *J, int b, int h, int g, int r,
+                               const int32_t *keys, int64_t nk, double *s, double *o,
+                               double *lse);
+
 /* One query row: the definition written out.
  *   K_set = { k : floor(k / blk) in T_{b,g}, k <= p }
  *   s_k   = scale * sum_d Q[b,h,r,d] K[b,g,k,d]
@@ -119,7 +125,7 @@ typedef struct {
  *   O[d]  = sum_{k in K_set} exp(s_k - LSE) V[b,g,k,d]                    */
 static int attention_row(const attn_job *J, int64_t flat, double *s, int32_t *keys,
                          double *o, double *lse) {
-    const int C = J->C, D = J->D, blk = J->blk;
+    const int C = J->C, blk = J->blk;
     const int r = (int)(flat % C);
     const int h = (int)((flat / C) % J->H_q);
     const int b = (int)(flat / ((int64_t)C * J->H_q));
@@ -127,6 +133,23 @@ static int attention_row(const attn_job *J, int64_t flat, double *s, int32_t *ke
     const int g = h / G;
     const int64_t p = (int64_t)J->chunk_start[b] + r;
     const int nKVmax = J->L_max / blk;
+
+    int64_t nk = 0;
+    if (J->tile_mask) {
+        /* Per-tile block-sparse baseline: row r of head h uses only the blocks
+         * its own Q-block i = floor(r / blk) selected in its own mask row,
+         *   K_set = { k : M[b,h,i,floor(k / blk)] != 0, k <= p }.         */
+        const uint8_t *mrow =
+            J->tile_mask + (((size_t)b * J->H_q + h) * J->nQ + r / blk) * (size_t)nKVmax;
+        for (int j = 0; j < nKVmax; ++j) {
+            if (mrow[j] == 0) continue;
+            for (int c = 0; c < blk; ++c) {
+                const int64_t k = (int64_t)j * blk + c;
+                if (k <= p) keys[nk++] = (int32_t)k;
+            }
+        }
+        return attention_over_keys(J, b, h, g, r, keys, nk, s, o, lse);
+    }
 
     int n_entries;
     const int32_t *T = NULL;
@@ -138,7 +161,6 @@ static int attention_row(const attn_job *J, int64_t flat, double *s, int32_t *ke
         n_entries = (J->chunk_start[b] + C + blk - 1) / blk;  /* nKV_b */
     }
 
-    int64_t nk = 0;
     for (int t = 0; t < n_entries; ++t) {
         const int j = T ? T[t] : t;
         if (j < 0 || j >= nKVmax) return ORACLE_ETABLE;
@@ -147,7 +169,16 @@ static int attention_row(const attn_job *J, int64_t flat, double *s, int32_t *ke
             if (k <= p) keys[nk++] = (int32_t)k;
         }
     }
+    return attention_over_keys(J, b, h, g, r, keys, nk, s, o, lse);
+}
 
+/* Softmax attention of query row (b, h, r) over the key positions keys[0, nk)
+ * of KV head g, in fp64: s_k = scale * q . K[k]; LSE = log sum exp(s_k)
+ * (max-subtracted); O = sum exp(s_k - LSE) V[k]. No key: O = 0, LSE = -inf. */
+static int attention_over_keys(const attn_job *J, int b, int h, int g, int r,
+                               const int32_t *keys, int64_t nk, double *s, double *o,
+                               double *lse) {
+    const int C = J->C, D = J->D;
     const uint16_t *q = J->Q + (((size_t)b * J->H_q + h) * C + r) * D;
     const uint16_t *Kbg = J->K + ((size_t)b * J->H_kv + g) * (size_t)J->L_max * D;
     const uint16_t *Vbg = J->V + ((size_t)b * J->H_kv + g) * (size_t)J->L_max * D;
@@ -208,15 +239,16 @@ static void *attn_worker(void *arg) {
  * dense reference (every block of the sequence's visible length).
  * Writes O (fp64, [n_rows, D]) and LSE (fp64, [n_rows]).
  */
-int oracle_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
-                          const int32_t *tables, const int32_t *counts,
-                          const int32_t *chunk_start, int B, int H_q, int H_kv, int C,
-                          int L_max, int D, int blk, double scale, const int64_t *rows,
-                          int64_t n_rows, double *O, double *LSE, int n_threads) {
+static int run_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                    const int32_t *tables, const int32_t *counts, const uint8_t *tile_mask,
+                    int nQ, const int32_t *chunk_start, int B, int H_q, int H_kv, int C,
+                    int L_max, int D, int blk, double scale, const int64_t *rows,
+                    int64_t n_rows, double *O, double *LSE, int n_threads) {
     if (!Q || !K || !V || !chunk_start || !O || !LSE || B <= 0 || H_q <= 0 || H_kv <= 0 ||
         H_q % H_kv != 0 || C <= 0 || L_max <= 0 || D <= 0 || blk <= 0 || L_max % blk != 0)
         return ORACLE_EINVAL;
     if (tables && !counts) return ORACLE_EINVAL;
+    if (tile_mask && (nQ <= 0 || (int64_t)nQ * blk < C)) return ORACLE_EINVAL;
     for (int b = 0; b < B; ++b)
         if (chunk_start[b] < 0 || (int64_t)chunk_start[b] + C > L_max)
             return ORACLE_EINVAL;
@@ -238,6 +270,7 @@ int oracle_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *
         attn_job *J = &jobs[w];
         J->Q = Q; J->K = K; J->V = V;
         J->tables = tables; J->counts = counts; J->chunk_start = chunk_start;
+        J->tile_mask = tile_mask; J->nQ = nQ;
         J->B = B; J->H_q = H_q; J->H_kv = H_kv; J->C = C; J->L_max = L_max;
         J->D = D; J->blk = blk; J->scale = scale;
         J->rows = rows; J->n_rows = n_rows; J->O = O; J->LSE = LSE;
@@ -267,6 +300,70 @@ int oracle_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *
     free(jobs);
     free(tid);
     return status;
+}
+
+int oracle_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                          const int32_t *tables, const int32_t *counts,
+                          const int32_t *chunk_start, int B, int H_q, int H_kv, int C,
+                          int L_max, int D, int blk, double scale, const int64_t *rows,
+                          int64_t n_rows, double *O, double *LSE, int n_threads) {
+    return run_rows(Q, K, V, tables, counts, NULL, 0, chunk_start, B, H_q, H_kv, C, L_max, D,
+                    blk, scale, rows, n_rows, O, LSE, n_threads);
+}
+
+/*
+ * Per-tile block-sparse attention (the ablation baseline the pages set
+ * against the Block-Union path: every head and Q-block keeps its own mask
+ * row, no union). mask: uint8 [B, H_q, nQ, L_max / blk]; everything else as
+ * in oracle_attention_rows.
+ */
+int oracle_attention_tile_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                               const uint8_t *mask, int nQ, const int32_t *chunk_start, int B,
+                               int H_q, int H_kv, int C, int L_max, int D, int blk,
+                               double scale, const int64_t *rows, int64_t n_rows, double *O,
+                               double *LSE, int n_threads) {
+    if (!mask) return ORACLE_EINVAL;
+    return run_rows(Q, K, V, NULL, NULL, mask, nQ, chunk_start, B, H_q, H_kv, C, L_max, D,
+                    blk, scale, rows, n_rows, O, LSE, n_threads);
+}
+
+/*
+ * Span tables for the per-tile path. The chunk's Q-blocks are taken in spans
+ * of `span` consecutive Q-blocks (the last span may be short); for each
+ * (b, h, span) the table lists, ascending, every KV block j that some
+ * Q-block of the span selects, as the entry
+ *     j | (bit u set iff Q-block span * span_index + u selects j) << 24,
+ * padded with -1; counts[b, h, span] is the number of entries. Shapes:
+ * tables int32 [B, H_q, nS, nKVmax], counts int32 [B, H_q, nS], nS =
+ * ceil(nQ / span). Requires nKVmax < 2^24 and 1 <= span <= 7.
+ */
+int oracle_tile_span_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int span,
+                            int32_t *tables, int32_t *counts) {
+    if (!mask || !tables || !counts || B <= 0 || H_q <= 0 || nQ <= 0 || nKVmax <= 0 ||
+        nKVmax >= (1 << 24) || span < 1 || span > 7)
+        return ORACLE_EINVAL;
+    const int nS = (nQ + span - 1) / span;
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H_q; ++h) {
+            for (int sp = 0; sp < nS; ++sp) {
+                const size_t item = ((size_t)b * H_q + h) * nS + sp;
+                int32_t *T = tables + item * nKVmax;
+                int n = 0;
+                for (int j = 0; j < nKVmax; ++j) {
+                    int bits = 0;
+                    for (int u = 0; u < span; ++u) {
+                        const int i = sp * span + u;
+                        if (i < nQ && mask[(((size_t)b * H_q + h) * nQ + i) * nKVmax + j] != 0)
+                            bits |= 1 << u;
+                    }
+                    if (bits) T[n++] = j | (bits << 24);
+                }
+                counts[item] = n;
+                for (int t = n; t < nKVmax; ++t) T[t] = -1;
+            }
+        }
+    }
+    return ORACLE_OK;
 }
 
 /* Number of (row, key) pairs the attention above touches, per row list: the

@@ -75,11 +75,17 @@ def _sdpa_masked(Q, K, V, allowed, scale):
     safe = allowed.clone()
     safe[..., 0] |= empty  # keep softmax finite; overwritten below
     O = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=safe, scale=scale)
-    logits = (q @ k.transpose(-1, -2)) * scale
-    LSE = torch.logsumexp(logits.masked_fill(~safe, float("-inf")), dim=-1)
-    O[empty] = 0.0
-    LSE[empty] = float("-inf")
-    return O.numpy(), LSE.numpy()
+    # LSE in numpy: torch's CPU logsumexp was seen to return a value off by
+    # ~2e-10 (relative) on rare first calls in a process.
+    logits = np.einsum("bhrd,bhkd->bhrk", q.numpy(), k.numpy()) * scale
+    logits = np.where(safe.numpy(), logits, -np.inf)
+    mx = logits.max(axis=-1, keepdims=True)
+    LSE = (mx + np.log(np.exp(logits - mx).sum(axis=-1, keepdims=True)))[..., 0]
+    O = O.numpy()
+    e = empty.numpy()
+    O[e] = 0.0
+    LSE[e] = -np.inf
+    return O, LSE
 
 
 def _causal_allowed(B, H_q, C, L, chunk_start):
@@ -414,3 +420,96 @@ def test_visible_pair_count():
     assert n == C * cs + C * (C + 1) // 2
     # the 128K / 2048 chunk dense count quoted for the LLaMA-8B shape
     assert 2048 * 131072 + 2048 * 2049 // 2 == 270_533_632
+
+
+# ------------------------------------------------ per-tile block-sparse path
+
+def _tile_allowed(mask, B, H_q, C, L, blk, cs):
+    """allowed[b, h, r, k]: block (r // blk, k // blk) selected by head h and
+    key k causally visible from position cs[b] + r (token-level expansion of
+    the block mask, built with plain indexing)."""
+    m = torch.as_tensor(mask).bool()
+    rows = torch.arange(C) // blk
+    keys = torch.arange(L) // blk
+    tile = m[:, :, rows][:, :, :, keys]  # [B, H_q, C, L]
+    return tile & _causal_allowed(B, H_q, C, L, cs)
+
+
+@pytest.mark.parametrize("cfg", [
+    # B, H_q, H_kv, D, blk, C, L_max, chunk_start, density
+    (1, 4, 1, 16, 8, 24, 64, (16,), 0.3),
+    (2, 6, 2, 8, 4, 12, 40, (0, 20), 0.5),
+    (2, 4, 2, 32, 8, 32, 96, (40, 8), 0.2),
+])
+def test_tile_attention_equals_sdpa_with_expanded_block_mask(cfg):
+    """Per-tile block-sparse attention is SDPA with the token-level mask that
+    the per-head per-Q-block block mask expands to (causal on top)."""
+    B, H_q, H_kv, D, blk, C, L, cs, dens = cfg
+    rng = np.random.default_rng(sum(cfg[:7]))
+    nQ, nK = C // blk, L // blk
+    mask = _rand_mask(rng, B, H_q, nQ, nK, dens)
+    Q, K, V = _rand_qkv(7 + B, B, H_q, H_kv, C, L, D)
+    scale = 0.9 / math.sqrt(D)
+    O, LSE = oracle.attention_tile(Q, K, V, cs, blk, mask, scale=scale)
+    Oref, LSEref = _sdpa_masked(Q, K, V, _tile_allowed(mask, B, H_q, C, L, blk, cs), scale)
+    np.testing.assert_allclose(O, Oref, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(LSE, LSEref, rtol=1e-10, atol=1e-10)
+    # some rows see no key at these densities: the convention O = 0, LSE = -inf
+    empty = ~_tile_allowed(mask, B, H_q, C, L, blk, cs).any(dim=-1).numpy()
+    assert np.all(O[empty] == 0.0) and np.all(np.isneginf(LSE[empty]))
+
+
+def test_tile_attention_on_union_closed_mask_equals_block_union_attention():
+    """When every head and Q-block of a group selects exactly the group's
+    union, the per-tile path and the Block-Union path attend to the same keys."""
+    rng = np.random.default_rng(11)
+    B, H_q, H_kv, D, blk, C, L = 2, 4, 2, 16, 8, 32, 96
+    cs = (48, 16)
+    G = H_q // H_kv
+    U = (rng.random((B, H_kv, L // blk)) < 0.4).astype(np.uint8)
+    mask = np.repeat(U, G, axis=1)[:, :, None, :].repeat(C // blk, axis=2)
+    T, cnt, _, _ = oracle.block_tables(mask, G)
+    Q, K, V = _rand_qkv(5, B, H_q, H_kv, C, L, D)
+    O1, L1 = oracle.attention_tile(Q, K, V, cs, blk, mask)
+    O2, L2 = oracle.attention(Q, K, V, cs, blk, T, cnt)
+    np.testing.assert_array_equal(np.isneginf(L1), np.isneginf(L2))
+    fin = ~np.isneginf(L2)
+    np.testing.assert_allclose(O1, O2, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(L1[fin], L2[fin], rtol=1e-12, atol=1e-12)
+
+
+def test_tile_attention_all_ones_is_dense_causal():
+    B, H_q, H_kv, D, blk, C, L, cs = 1, 4, 2, 16, 8, 24, 64, (24,)
+    Q, K, V = _rand_qkv(3, B, H_q, H_kv, C, L, D)
+    mask = np.ones((B, H_q, C // blk, L // blk), np.uint8)
+    O, LSE = oracle.attention_tile(Q, K, V, cs, blk, mask)
+    Oref, LSEref = _sdpa_masked(Q, K, V, _causal_allowed(B, H_q, C, L, cs), 1 / math.sqrt(D))
+    np.testing.assert_allclose(O, Oref, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(LSE, LSEref, rtol=1e-10, atol=1e-10)
+
+
+@pytest.mark.parametrize("span", [1, 2, 3, 4])
+def test_tile_span_tables_round_trip_and_order(span):
+    """The span tables encode the mask losslessly: decoding every entry's
+    bits gives back exactly the nonzero pattern of every mask row; entries are
+    strictly ascending, each has at least one bit, the tail is -1."""
+    rng = np.random.default_rng(100 + span)
+    B, H_q, nQ, nK = 2, 3, 7, 40
+    mask = (rng.random((B, H_q, nQ, nK)) < 0.25).astype(np.uint8) * rng.integers(1, 255, (B, H_q, nQ, nK), dtype=np.uint8)
+    T, cnt = oracle.tile_span_tables(mask, span)
+    nS = -(-nQ // span)
+    assert T.shape == (B, H_q, nS, nK) and cnt.shape == (B, H_q, nS)
+    rebuilt = np.zeros((B, H_q, nS * span, nK), bool)
+    for b in range(B):
+        for h in range(H_q):
+            for s in range(nS):
+                n = cnt[b, h, s]
+                e = T[b, h, s, :n].astype(np.int64)
+                j, bits = e & ((1 << 24) - 1), e >> 24
+                assert np.all(np.diff(j) > 0) and np.all(bits > 0)
+                assert np.all(bits < (1 << span))
+                assert np.all(T[b, h, s, n:] == -1)
+                for u in range(span):
+                    rebuilt[b, h, s * span + u, j[(bits >> u) & 1 == 1]] = True
+    np.testing.assert_array_equal(rebuilt[:, :, :nQ], mask != 0)
+    assert not rebuilt[:, :, nQ:].any()
