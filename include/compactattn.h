@@ -161,6 +161,52 @@ int ca_compacted_chunk_attention(const void *Q, const void *Kc, const void *Vc,
                                  void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Per-tile block-sparse ablation (pages: "Problem", block-sparse kernels that
+ * execute the 2D mask directly in the Q << KV regime, and the efficiency
+ * ablation under "Experimental results"): every query head and Q-block
+ * attends to its own selected blocks, with no Q-block or intra-group union:
+ *   K_set(b, h, r) = { k : mask[b, h, r / blk, k / blk] != 0, k <= p }.
+ *
+ * Q-blocks per span: the per-tile kernel processes 256 chunk rows of one head
+ * per work item, so its tables group each head's Q-blocks in spans of
+ * 256 / blk. Returns that number (2 for blk 128, 4 for blk 64), 0 if blk is
+ * unsupported.
+ */
+int ca_tile_span(int blk);
+
+/*
+ * Per-tile ablation, step 1: span tables from the mask. For each (b, h,
+ * span s), nS = ceil(nQ / span) spans with span = ca_tile_span(blk):
+ *   tables[b, h, s, 0 : counts[b, h, s]] = ascending KV blocks j that some
+ *   Q-block i = span * s + u (u < span, i < nQ) selects, each stored as
+ *   j | (bit u set iff mask[b, h, span * s + u, j] != 0) << 24;
+ *   tables[b, h, s, counts[b, h, s] :] = -1.
+ * mask    device uint8 [B, H_q, nQ, nKVmax], nonzero = selected
+ * tables  device int32 [B, H_q, nS, nKVmax] (written), counts int32
+ *         [B, H_q, nS] (written); caller-owned, 4-byte aligned.
+ * Requires nKVmax < 2^24. Errors: CA_ERR_INVALID_ARG, CA_ERR_SHAPE,
+ * CA_ERR_ALIGN, CA_ERR_UNSUPPORTED (blk), CA_ERR_CUDA.
+ */
+int ca_build_tile_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int blk,
+                         int32_t *tables, int32_t *counts, void *stream);
+
+/*
+ * Per-tile ablation, step 2: attention over the span tables of
+ * ca_build_tile_tables, read in place from the cache. A work item holds two
+ * 128-row tiles of one query head and walks its span's table; a tile's rows
+ * skip (P = 0) every block their own Q-block did not select, so the result is
+ * per-tile block-sparse attention. Each head loads its own K/V blocks (no
+ * sharing across the GQA group). Arguments and errors as ca_chunk_attention,
+ * with tables / counts shaped [B, H_q, nS, L_max / blk] / [B, H_q, nS],
+ * nS = ceil(C / 256) (the mask had nQ = ceil(C / blk) Q-blocks); requires
+ * L_max / blk < 2^24.
+ */
+int ca_tile_chunk_attention(const void *Q, const void *K, const void *V, const int32_t *tables,
+                            const int32_t *counts, const int32_t *chunk_start, int B, int H_q,
+                            int H_kv, int C, int L_max, int D, int blk, float scale, void *O,
+                            float *LSE, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * ca_chunk_attention without a caller workspace, for callers that cannot
  * allocate device memory when they run attention (an engine whose device
  * memory is sized once at start-up, code inside a fixed memory pool, a host

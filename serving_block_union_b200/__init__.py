@@ -69,6 +69,9 @@ EXPORTED_SYMBOLS = (
     "ca_selftest_bounded_wait",
     "ca_compact_kv_blocks",
     "ca_compacted_chunk_attention",
+    "ca_tile_span",
+    "ca_build_tile_tables",
+    "ca_tile_chunk_attention",
 )
 
 
@@ -117,6 +120,13 @@ def load_library():
         lib.ca_compacted_chunk_attention.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P,
                                                      P, P, S, P]
         lib.ca_compacted_chunk_attention.restype = I
+        lib.ca_tile_span.argtypes = [I]
+        lib.ca_tile_span.restype = I
+        lib.ca_build_tile_tables.argtypes = [P, I, I, I, I, I, P, P, P]
+        lib.ca_build_tile_tables.restype = I
+        lib.ca_tile_chunk_attention.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P, P, P,
+                                                S, P]
+        lib.ca_tile_chunk_attention.restype = I
         _lib = lib
         return lib
 
@@ -401,4 +411,75 @@ def compacted_chunk_attention(Q: torch.Tensor, Kc: torch.Tensor, Vc: torch.Tenso
         blk, float(scale), _ptr(O), _ptr(LSE), _ptr(workspace), workspace.numel(),
         _stream_handle(stream, Q.device))
     _check("ca_compacted_chunk_attention", st)
+    return O, LSE
+
+
+# ------------------------------------------- per-tile block-sparse ablation
+
+def tile_span(blk: int) -> int:
+    """Q-blocks per span of the per-tile path's tables (256 chunk rows)."""
+    n = int(load_library().ca_tile_span(int(blk)))
+    if n == 0:
+        raise ValueError(f"unsupported block size {blk}")
+    return n
+
+
+def build_tile_tables(mask: torch.Tensor, blk: int, tables: Optional[torch.Tensor] = None,
+                      counts: Optional[torch.Tensor] = None,
+                      stream: Optional[torch.cuda.Stream] = None):
+    """Span tables of the per-tile block-sparse path from a uint8 / bool mask
+    ``[B, H_q, nQ, nKVmax]``: per (b, h, span of ``tile_span(blk)`` Q-blocks)
+    the ascending KV blocks any Q-block of the span selects, each entry
+    ``j | bits << 24`` (bit u: Q-block ``span*s + u`` selects j), tail -1.
+    Returns ``(tables int32 [B, H_q, nS, nKVmax], counts int32 [B, H_q, nS])``."""
+    if mask.dtype == torch.bool:
+        mask = mask.view(torch.uint8)
+    _need(mask, "mask", torch.uint8, 4)
+    B, H_q, nQ, nK = mask.shape
+    span = tile_span(blk)
+    nS = -(-nQ // span)
+    dev = mask.device
+    if tables is None:
+        tables = torch.empty((B, H_q, nS, nK), dtype=torch.int32, device=dev)
+    if counts is None:
+        counts = torch.empty((B, H_q, nS), dtype=torch.int32, device=dev)
+    _need(tables, "tables", torch.int32, 4)
+    _need(counts, "counts", torch.int32, 3)
+    if tuple(tables.shape) != (B, H_q, nS, nK) or tuple(counts.shape) != (B, H_q, nS):
+        raise ValueError(f"tables must be {(B, H_q, nS, nK)}, counts {(B, H_q, nS)}")
+    st = load_library().ca_build_tile_tables(_ptr(mask), B, H_q, nQ, nK, int(blk), _ptr(tables),
+                                             _ptr(counts), _stream_handle(stream, dev))
+    _check("ca_build_tile_tables", st)
+    return tables, counts
+
+
+def tile_chunk_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, tables: torch.Tensor,
+                         counts: torch.Tensor, chunk_start: Sequence[int],
+                         scale: Optional[float] = None, O: Optional[torch.Tensor] = None,
+                         LSE: Optional[torch.Tensor] = None,
+                         workspace: Optional[torch.Tensor] = None,
+                         stream: Optional[torch.cuda.Stream] = None
+                         ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-tile block-sparse chunk attention over build_tile_tables' span
+    tables: row r of head h attends to the keys k <= chunk_start[b] + r of the
+    blocks its own Q-block selected (no union), read in place from the cache."""
+    _need(tables, "tables", torch.int32, 4)
+    _need(counts, "counts", torch.int32, 3)
+    nK = tables.shape[-1]
+    L_max = K.shape[2]
+    if nK <= 0 or L_max % nK:
+        raise ValueError("tables' last dim must divide L_max (it is L_max / blk)")
+    blk = L_max // nK
+    B, H_q, H_kv, C, L_max, D, O, LSE, workspace = _attn_common(Q, K, V, O, LSE, workspace, blk)
+    nS = -(-C // 256)
+    if tuple(tables.shape[:3]) != (B, H_q, nS) or tuple(counts.shape) != (B, H_q, nS):
+        raise ValueError(f"tables must be {(B, H_q, nS, nK)}, counts {(B, H_q, nS)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    cs = _chunk_start_host(chunk_start, B)
+    st = load_library().ca_tile_chunk_attention(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(tables), _ptr(counts), cs, B, H_q, H_kv, C, L_max, D,
+        blk, float(scale), _ptr(O), _ptr(LSE), _ptr(workspace), workspace.numel(),
+        _stream_handle(stream, Q.device))
+    _check("ca_tile_chunk_attention", st)
     return O, LSE

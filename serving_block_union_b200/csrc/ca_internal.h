@@ -38,6 +38,18 @@ struct AttnArgs {
 constexpr int kModeTables = 0;
 constexpr int kModeDense = 1;
 constexpr int kModeCompact = 2;
+// Per-tile block-sparse ablation: one work item per (b, query head, 256 chunk
+// rows), walking that head's span table (entries j | Q-block bits << 24).
+constexpr int kModePerTile = 3;
+
+// Chunk rows of one per-tile work item (two 128-row tiles of one head); the
+// span tables group a head's Q-blocks by it.
+constexpr int kTileItemRows = 256;
+// Low bits of a span-table entry that hold the KV block index.
+constexpr int kSpanEntryBits = 24;
+
+int launch_tile_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int span,
+                       int32_t *tables, int32_t *counts, cudaStream_t stream);
 
 int launch_chunk_attention(const AttnArgs &a, int mode, cudaStream_t stream);
 

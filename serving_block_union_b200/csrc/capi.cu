@@ -141,6 +141,38 @@ int ca_compacted_chunk_attention(const void *Q, const void *Kc, const void *Vc,
     return ca::launch_chunk_attention(a, ca::kModeCompact, static_cast<cudaStream_t>(stream));
 }
 
+int ca_tile_span(int blk) {
+    return (blk == 64 || blk == 128) ? ca::kTileItemRows / blk : 0;
+}
+
+int ca_build_tile_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int blk,
+                         int32_t *tables, int32_t *counts, void *stream) {
+    if (!mask || !tables || !counts) return CA_ERR_INVALID_ARG;
+    if (B <= 0 || H_q <= 0 || nQ <= 0 || nKVmax <= 0 || blk <= 0) return CA_ERR_INVALID_ARG;
+    const int span = ca_tile_span(blk);
+    if (span == 0) return CA_ERR_UNSUPPORTED;
+    if (nKVmax >= (1 << ca::kSpanEntryBits)) return CA_ERR_SHAPE;
+    const long long nS = (nQ + span - 1) / span;
+    if ((long long)B * H_q * nQ * nKVmax >= (1LL << 40)) return CA_ERR_SHAPE;
+    if ((long long)B * H_q * nS >= (1LL << 31)) return CA_ERR_SHAPE;
+    if (!aligned(tables, 4) || !aligned(counts, 4)) return CA_ERR_ALIGN;
+    return ca::launch_tile_tables(mask, B, H_q, nQ, nKVmax, span, tables, counts,
+                                  static_cast<cudaStream_t>(stream));
+}
+
+int ca_tile_chunk_attention(const void *Q, const void *K, const void *V, const int32_t *tables,
+                            const int32_t *counts, const int32_t *chunk_start, int B, int H_q,
+                            int H_kv, int C, int L_max, int D, int blk, float scale, void *O,
+                            float *LSE, void *workspace, size_t workspace_bytes, void *stream) {
+    const int st = check_attention(Q, K, V, tables, counts, false, chunk_start, B, H_q, H_kv, C,
+                                   L_max, D, blk, scale, O, LSE, workspace, workspace_bytes);
+    if (st != CA_OK) return st;
+    if (L_max / blk >= (1 << ca::kSpanEntryBits)) return CA_ERR_SHAPE;
+    ca::AttnArgs a{Q, K, V, tables, counts, chunk_start, B, H_q, H_kv, C, L_max, D, blk,
+                   scale, O, LSE, workspace};
+    return ca::launch_chunk_attention(a, ca::kModePerTile, static_cast<cudaStream_t>(stream));
+}
+
 int ca_read_device_status(const void *workspace, void *stream) {
     if (!workspace) return CA_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -138,15 +138,23 @@ struct Layout {
     static_assert(kDynamic <= kSmemBudget, "shared memory budget exceeded");
 };
 
+// KV block index of a table entry (span-table entries carry Q-block bits
+// above kSpanEntryBits).
+template <bool SPAN>
+__device__ __forceinline__ int block_of(int e) {
+    return SPAN ? (e & ((1 << kSpanEntryBits) - 1)) : e;
+}
+
 // Entries of the ascending prefix T[0, n) that are <= bound; warp-cooperative
 // (all 32 lanes), scanning windows of 32 from the end (the answer is normally
 // in the last window: only blocks inside the chunk can lie past the bound).
+template <bool SPAN>
 __device__ __forceinline__ int count_le(const int32_t *T, int n, int bound, int lane) {
     int hi = n;
     while (hi > 0) {
         const int lo = hi > 32 ? hi - 32 : 0;
         const int idx = lo + lane;
-        const int v = idx < hi ? __ldg(T + idx) : 0;
+        const int v = idx < hi ? block_of<SPAN>(__ldg(T + idx)) : 0;
         const unsigned gt = __ballot_sync(0xffffffffu, idx < hi && v > bound);
         const int ngt = __popc(gt);
         if (ngt < hi - lo) return hi - ngt;
@@ -191,6 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     using L = Layout<D, BLK>;
     constexpr bool DENSE = MODE == kModeDense;
     constexpr bool COMPACT = MODE == kModeCompact;  // K/V block t sits at row t * BLK
+    constexpr bool PERTILE = MODE == kModePerTile;  // one head per tile, span tables
     constexpr int NST = L::kStages;
     constexpr int DCH = D / 64;  // 64-element (128-byte) sub-tiles along D
     constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, BLK, false);
@@ -219,12 +228,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work item
-    const int per_b = P.H_kv * P.n_pairs;
+    // ---- work item: (b, pair, unit), the unit a KV group, or a query head in
+    // the per-tile mode
+    const int units = PERTILE ? P.H_q : P.H_kv;
+    const int per_b = units * P.n_pairs;
     const int b = P.b_order[blockIdx.x / per_b];
     const int rem = blockIdx.x % per_b;
-    const int pair = rem / P.H_kv;
-    const int g = rem % P.H_kv;
+    const int pair = rem / units;
+    const int unit = rem % units;
+    const int g = PERTILE ? unit / P.G : unit;     // KV head
+    const int head0 = PERTILE ? unit : g * P.G;  // query head of packed row 0
     const int cs = P.chunk_start[b];
     const int R = P.R;
     const int r0 = pair * 2 * R;
@@ -274,14 +287,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         n_eff = jlast + 1;
         n_full = jfull + 1 > 0 ? jfull + 1 : 0;
     } else {
-        int cnt = __ldg(P.counts + b * P.H_kv + g);
+        const size_t trow = PERTILE ? ((size_t)b * P.H_q + unit) * P.n_pairs + pair
+                                    : (size_t)b * P.H_kv + g;
+        int cnt = __ldg(P.counts + trow);
         if (cnt < 0 || cnt > P.nKVmax) {
             if (threadIdx.x == 0) atomicOr(P.status, kDevErrTable);
             cnt = 0;
         }
-        T = P.tables + ((size_t)b * P.H_kv + g) * P.nKVmax;
-        n_eff = count_le(T, cnt, jlast, lane);
-        n_full = count_le(T, n_eff, jfull, lane);
+        T = P.tables + trow * P.nKVmax;
+        n_eff = count_le<PERTILE>(T, cnt, jlast, lane);
+        n_full = count_le<PERTILE>(T, n_eff, jfull, lane);
     }
 
     // Role code sits inside the branch that re-sized its registers, so the
@@ -298,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int t = 0; t < 2; ++t)
                     for (int dc = 0; dc < DCH; ++dc)
                         tma_load_3d(smem + L::kQOff + t * L::kQTile + dc * (kTileM * 128), &tmQ,
-                                    q_full, dc * 64, r0 + t * R, b * P.H_q + g * P.G);
+                                    q_full, dc * 64, r0 + t * R, b * P.H_q + head0);
             }
             q_issued = true;
             int prev_last = -1;
@@ -306,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int w0 = 0; w0 < n_eff && ok; w0 += 32) {
                 const int jj = w0 + lane;
                 const int nwin = min(32, n_eff - w0);
-                int jb = DENSE ? jj : (lane < nwin ? __ldg(T + jj) : 0);
+                int jb = DENSE ? jj : (lane < nwin ? block_of<PERTILE>(__ldg(T + jj)) : 0);
                 if (!DENSE) {
                     int prv = __shfl_up_sync(0xffffffffu, jb, 1);
                     if (lane == 0) prv = prev_last;
@@ -460,7 +475,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int r = r0 + t * R + (m % R);
         const bool valid = r < P.C;
         const int p = cs + r;
-        const int h = g * P.G + h_local;
+        const int h = head0 + h_local;
+        // per-tile mode: bit of this row's Q-block in the span-table entries
+        // (the 32 rows of a warp share one Q-block, so it is warp-uniform)
+        const int member_shift = kSpanEntryBits + (r / BLK - r0 / BLK);
         const uint32_t lane_base = static_cast<uint32_t>(qw * 32) << 16;
         const uint32_t tS = tmem + lane_base + t * 128;
         const uint32_t tO = tmem + lane_base + 256 + t * 128 + hf * DW;
@@ -492,6 +510,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
+            int e_j = 0;
+            if (PERTILE) e_j = __ldg(T + j);
+            if (PERTILE && ((e_j >> member_shift) & 1) == 0) {
+                // block not selected by this row's Q-block: P = 0, the running
+                // max and sum are unchanged
+                uint32_t zero[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) zero[i] = 0u;
+#pragma unroll
+                for (int cl = 0; cl < CPW; ++cl) {
+                    constexpr int CK = L::kPChunkKeys;
+                    const int c = hf * CPW + cl;
+#pragma unroll
+                    for (int q = 0; q < CK / 32; ++q) tmem_st16(tS + c * (CK / 2) + q * 16, zero);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    mbar_arrive_lane0(p_full + t * NPC + c, lane);
+                }
+                continue;
+            }
             float s[CW];
             {
                 uint32_t v[CW];
@@ -500,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < CW; ++i) s[i] = __uint_as_float(v[i]);
             }
             if (j >= n_full) {
-                int jb = DENSE ? j : __ldg(T + j);
+                int jb = DENSE ? j : (PERTILE ? block_of<true>(e_j) : __ldg(T + j));
                 jb = min(max(jb, 0), P.nKVmax);  // only matters for a flagged, invalid table
                 const int lim = p - jb * BLK - hf * CW;  // columns c <= lim are visible
 #pragma unroll
@@ -695,12 +734,13 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
     if (kRegSplit && num_regs != kLaunchRegs) return CA_ERR_UNSUPPORTED;
 
     const int G = a.H_q / a.H_kv;
-    const int R = kTileM / G;
+    const int pack = MODE == kModePerTile ? 1 : G;  // query heads packed into a tile
+    const int R = kTileM / pack;
     const int n_tiles = (a.C + R - 1) / R;
     const int n_pairs = (n_tiles + 1) / 2;
 
     CUtensorMap tq, tk, tv;
-    if (!encode_3d(&tq, a.Q, (uint64_t)D, (uint64_t)a.C, (uint64_t)a.B * a.H_q, 64, R, G) ||
+    if (!encode_3d(&tq, a.Q, (uint64_t)D, (uint64_t)a.C, (uint64_t)a.B * a.H_q, 64, R, pack) ||
         !encode_3d(&tk, a.K, (uint64_t)D, (uint64_t)a.L_max, (uint64_t)a.B * a.H_kv, 64, BLK, 1) ||
         !encode_3d(&tv, a.V, (uint64_t)D, (uint64_t)a.L_max, (uint64_t)a.B * a.H_kv, 64, BLK, 1))
         return CA_ERR_CUDA;
@@ -737,7 +777,8 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
         P.chunk_start[i] = i < a.B ? a.chunk_start[i] : 0;
         P.b_order[i] = static_cast<unsigned char>(i < a.B ? order[i] : 0);
     }
-    const unsigned grid = static_cast<unsigned>(a.B * a.H_kv * n_pairs);
+    const int units = MODE == kModePerTile ? a.H_q : a.H_kv;
+    const unsigned grid = static_cast<unsigned>(a.B * units * n_pairs);
     kern<<<grid, kThreads, L::kDynamic, stream>>>(tq, tk, tv, P);
     return cudaGetLastError() == cudaSuccess ? CA_OK : CA_ERR_CUDA;
 }
@@ -749,6 +790,7 @@ int launch_chunk_attention(const AttnArgs &a, int mode, cudaStream_t stream) {
     if (a.D == D_ && a.blk == BLK_) {                                                 \
         if (mode == kModeDense) return launch_t<D_, BLK_, kModeDense>(a, stream);     \
         if (mode == kModeCompact) return launch_t<D_, BLK_, kModeCompact>(a, stream); \
+        if (mode == kModePerTile) return launch_t<D_, BLK_, kModePerTile>(a, stream); \
         return launch_t<D_, BLK_, kModeTables>(a, stream);                            \
     }
     CA_DISPATCH(128, 128)

@@ -113,6 +113,24 @@ def test_build_tables_host_checks(lib):
     assert f(A16, 0, 32, 16, 272, 4, A16, A16, None, None, None) == ca.CA_ERR_INVALID_ARG
 
 
+def test_tile_path_host_checks(lib):
+    assert lib.ca_tile_span(128) == 2 and lib.ca_tile_span(64) == 4
+    assert lib.ca_tile_span(32) == 0
+    f = lib.ca_build_tile_tables
+    assert f(None, 1, 32, 16, 272, 128, A16, A16, None) == ca.CA_ERR_INVALID_ARG
+    assert f(A16, 1, 32, 16, 272, 32, A16, A16, None) == ca.CA_ERR_UNSUPPORTED
+    assert f(A16, 1, 32, 16, 1 << 24, 128, A16, A16, None) == ca.CA_ERR_SHAPE
+    assert f(A16, 1, 32, 16, 272, 128, A_MIS, A16, None) == ca.CA_ERR_ALIGN
+    cs = (ctypes.c_int32 * 1)(32768)
+    g = lib.ca_tile_chunk_attention
+    assert g(A16, A16, A16, None, A16, cs, 1, 32, 8, 2048, 34816, 128, 128, 0.1, A16, A16, A16,
+             256, None) == ca.CA_ERR_INVALID_ARG
+    assert g(A16, A16, A16, A16, A16, cs, 1, 32, 8, 2048, 34800, 128, 128, 0.1, A16, A16, A16,
+             256, None) == ca.CA_ERR_SHAPE
+    assert g(A16, A16, A16, A16, A16, cs, 1, 32, 8, 2048, 34816, 96, 128, 0.1, A16, A16, A16,
+             256, None) == ca.CA_ERR_UNSUPPORTED
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     monkeypatch.setattr(ca, "_lib", None)

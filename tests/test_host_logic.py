@@ -30,6 +30,22 @@ def test_bench_visible_pairs_matches_oracle():
                                              wl.L_max, wl.blk)
 
 
+def test_bench_tile_visible_pairs_matches_token_count():
+    """Per-tile work count: the token-level expansion of the block mask, causal
+    on top, counted pair by pair."""
+    rng = np.random.default_rng(4)
+    B, H_q, blk, C, L = 2, 3, 8, 40, 128
+    cs = (56, 8)
+    nQ, nK = -(-C // blk), L // blk
+    mask = (rng.random((B, H_q, nQ, nK)) < 0.3).astype(np.uint8)
+    tok = np.repeat(np.repeat(mask != 0, blk, axis=2)[:, :, :C], blk, axis=3)
+    total = 0
+    for b in range(B):
+        causal = np.arange(L)[None, :] <= cs[b] + np.arange(C)[:, None]
+        total += int((tok[b] & causal[None]).sum())
+    assert bench.tile_visible_pairs(mask, cs, C, blk) == total
+
+
 def _poly_coeffs():
     src = open(os.path.join(ROOT, "serving_block_union_b200", "csrc", "sm100_ptx.cuh")).read()
     body = src[src.index("float exp2_poly(float x)"):]
