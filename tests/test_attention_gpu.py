@@ -119,7 +119,7 @@ def test_tiny_workload_tables_from_gpu_builder(cuda_ok):
 
 FULL = ["llama8b_32k", "llama8b_128k_d2", "llama8b_128k_d5", "llama8b_128k_d10",
         "llama8b_128k_d20", "llama8b_128k_noise", "batched", "full_prefill_c0",
-        "full_prefill_c1", "full_prefill_c31", "full_prefill_c63"]
+        "full_prefill_c1", "full_prefill_c31", "full_prefill_c63", "qwen3_30b_128k_d10"]
 
 
 def _poison_unselected(wl, K, V, T, c):

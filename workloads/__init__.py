@@ -39,6 +39,7 @@ __all__ = [
     "llama8b_128k",
     "batched",
     "full_prefill_chunk",
+    "qwen3_30b_128k",
     "by_name",
     "make_mask",
     "make_qkv",
@@ -137,6 +138,17 @@ def llama8b_128k(density: float = 0.10, noise: bool = False) -> Workload:
                     seed=200 + pct, mask_kind="stripes", density=density)
 
 
+def qwen3_30b_128k(density: float = 0.10) -> Workload:
+    """The 128K sweep's mask and sizes with a GQA group of 8: 32 query heads
+    over 4 KV heads, head dim 128 (the attention shape of the pages' second
+    model, Qwen3-30B-A3B; the pages do not print it). Eight heads' independent
+    stripes make the group union larger than at G = 4."""
+    pct = int(round(density * 100))
+    return Workload(f"qwen3_30b_128k_d{pct}", B=1, H_q=32, H_kv=4, D=128, blk=128,
+                    C=2048, L_max=131072 + 2048, chunk_start=(131072,),
+                    seed=300 + pct, mask_kind="stripes", density=density)
+
+
 def batched() -> Workload:
     """B=4 sequences with 16K/32K/64K/96K cached tokens and a 4096-token chunk;
     per-head density U(2%, 15%); heads of a group share only half of their
@@ -167,6 +179,8 @@ def by_name(name: str) -> Workload:
         return llama8b_128k(noise=True)
     if name == "batched":
         return batched()
+    if name.startswith("qwen3_30b_128k_d"):
+        return qwen3_30b_128k(int(name[len("qwen3_30b_128k_d"):]) / 100.0)
     if name.startswith("full_prefill_c"):
         return full_prefill_chunk(int(name[len("full_prefill_c"):]))
     raise KeyError(name)
