@@ -76,10 +76,16 @@ int ca_build_block_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVma
                           int32_t *tables, int32_t *counts, int32_t *indptr, int32_t *indices,
                           void *stream);
 
-/* Bytes of device workspace ca_chunk_attention / ca_dense_chunk_attention need
- * for these sizes (a status word plus scheduler state). Allocate it once,
- * 256-byte aligned and zero-filled; it can be reused by later calls on the
- * same stream. Returns 0 for invalid sizes. */
+/* Bytes of device workspace the attention entry points use for these sizes on
+ * the current device, for D <= 128: a 256-byte header (status word) plus room
+ * for the split of the last wave of work items (split-KV: when the items do
+ * not fill the SMs evenly, the remaining items' block lists are cut into
+ * segments run by separate CTAs; each writes a partial O and LSE, merged by
+ * the item's last CTA). Any workspace of at least 256 bytes is valid; one
+ * smaller than this value runs without the split. Allocate it once, 256-byte
+ * aligned and zero-filled, and reuse it for later calls on the same stream;
+ * after a call that reported a device error, zero it again. Returns 0 for
+ * invalid sizes. */
 size_t ca_workspace_bytes(int B, int H_q, int H_kv, int C, int blk);
 
 /*
@@ -105,7 +111,8 @@ size_t ca_workspace_bytes(int B, int H_q, int H_kv, int C, int blk);
  * counts  int32 [B, H_kv]
  * chunk_start  HOST int32 [B], 0 <= chunk_start[b], chunk_start[b] + C <= L_max
  * O       bf16 [B, H_q, C, D] (16-byte aligned), LSE fp32 [B, H_q, C] or NULL
- * workspace   >= ca_workspace_bytes(...) bytes, 256-byte aligned, zeroed once.
+ * workspace   >= 256 bytes (ca_workspace_bytes(...) to allow the last-wave
+ *         split), 256-byte aligned, zeroed once.
  * Supported: D in {64, 128}, blk in {64, 128}, G in {1, 2, 4, 8, 16},
  * 1 <= B <= 128, L_max % blk == 0.
  * Errors (host): CA_ERR_INVALID_ARG, CA_ERR_SHAPE, CA_ERR_ALIGN,
@@ -216,8 +223,10 @@ int ca_tile_chunk_attention(const void *Q, const void *K, const void *V, const i
  * Same arguments and results as ca_chunk_attention minus the workspace; it
  * allocates nothing (no cudaMalloc / cudaFree, no allocating library call).
  * The scratch it needs comes from a fixed 4096-byte array inside the library,
- * held by every GPU that loads the library until the process exits; sizes whose
- * workspace (ca_workspace_bytes) would exceed it return CA_ERR_WORKSPACE.
+ * held by every GPU that loads the library until the process exits. That
+ * holds the status word and header the kernels need at minimum, not the
+ * partial results of the last-wave split, so calls through this entry point
+ * always run unsplit (same results within rounding, sometimes slower).
  * The first call on each device looks up that device's copy of the array
  * (cudaGetSymbolAddress, with that device current), so make that first call
  * before any stream capture. Every call on a device shares the one array:

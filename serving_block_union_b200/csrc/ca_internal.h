@@ -29,6 +29,7 @@ struct AttnArgs {
     void *O;
     float *LSE;
     void *workspace;
+    size_t workspace_bytes;
 };
 
 // Attention kernel modes: walk the tables over the cache in place; every block
@@ -52,6 +53,78 @@ int launch_tile_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, 
                        int32_t *tables, int32_t *counts, cudaStream_t stream);
 
 int launch_chunk_attention(const AttnArgs &a, int mode, cudaStream_t stream);
+
+// ---- split of the last wave (split-KV with an LSE merge)
+//
+// One CTA runs one work item (two 128-row tiles against a block list) and one
+// CTA fits an SM, so n_items CTAs take ceil(n_items / SMs) waves and the last
+// wave can be mostly empty (256 items on 148 SMs: 1.73 waves of work in 2).
+// The plan keeps the full waves [0, n_first) whole and cuts each remaining
+// item's block list into `split` segments run by separate CTAs, choosing the
+// split that makes those segment waves shortest. Each segment CTA writes a
+// normalised fp32 partial O and its base-2 LSE to the workspace; the last of
+// an item's CTAs to finish merges them (workspace counters, no waiting).
+constexpr int kMaxSplit = 8;
+constexpr int kRowsPerItem = 256;     // packed rows of one item (two tiles)
+constexpr int kSplitMinBlocks = 64;   // items shorter than this are not split
+
+struct SplitPlan {
+    int n_items = 0, n_first = 0, split = 1;
+    size_t bytes = kWorkspaceHeader;  // workspace this plan needs
+    size_t lse_off = 0, o_off = 0;    // byte offsets of the partial LSE / O arrays
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Build-time overrides for measurements: CA_SPLIT_FORCE = S splits every
+// item outside the first full waves into S segments (1: never split);
+// CA_SPLIT_ALL = 1 splits every item (no unsplit waves).
+#ifndef CA_SPLIT_FORCE
+#define CA_SPLIT_FORCE 0
+#endif
+#ifndef CA_SPLIT_ALL
+#define CA_SPLIT_ALL 0
+#endif
+
+inline SplitPlan plan_split(int n_items, int num_sms, int D, bool allow) {
+    SplitPlan p;
+    p.n_items = p.n_first = n_items;
+    if (!allow || num_sms <= 0 || n_items <= 0) return p;
+    const int n_first = CA_SPLIT_ALL ? 0 : (n_items / num_sms) * num_sms;
+    const int n_rest = n_items - n_first;
+    if (n_rest == 0) return p;
+    int best_s = 1;
+    long long best_waves = 1, best_den = 1;  // last waves' length as a fraction
+    for (int s = 2; s <= kMaxSplit; ++s) {
+        const long long waves = ((long long)n_rest * s + num_sms - 1) / num_sms;
+        if (waves * best_den < best_waves * s) {  // waves / s < best
+            best_s = s;
+            best_waves = waves;
+            best_den = s;
+        }
+    }
+    if (CA_SPLIT_FORCE > 0) best_s = CA_SPLIT_FORCE < kMaxSplit ? CA_SPLIT_FORCE : kMaxSplit;
+    if (best_s == 1) return p;
+    const size_t rows = (size_t)n_rest * best_s * kRowsPerItem;
+    p.n_first = n_first;
+    p.split = best_s;
+    p.lse_off = kWorkspaceHeader + align256(4 * (size_t)n_rest);
+    p.o_off = p.lse_off + align256(4 * rows);
+    p.bytes = p.o_off + 4 * rows * (size_t)D;
+    return p;
+}
+
+// Work items of one attention launch: B * units * pairs, the unit a KV group
+// (G query heads packed per tile) or, in the per-tile mode, a query head.
+inline int attention_items(int B, int H_q, int H_kv, int C, bool per_tile) {
+    const int pack = per_tile ? 1 : H_q / H_kv;
+    const int R = 128 / pack;
+    const int n_pairs = ((C + R - 1) / R + 1) / 2;
+    return B * (per_tile ? H_q : H_kv) * n_pairs;
+}
+
+// SM count of the current device (cached per device; 148 if it cannot be read).
+int current_sm_count();
 
 // Copies the K and V blocks each table selects into compact buffers: block
 // tables[b,g,t] of the cache goes to rows [t * blk, (t + 1) * blk) of Kc / Vc.

@@ -42,7 +42,7 @@ int check_attention(const void *Q, const void *K, const void *V, const int32_t *
     if ((LSE && !aligned(LSE, 4)) || (tables && !aligned(tables, 4)) ||
         (counts && !aligned(counts, 4)))
         return CA_ERR_ALIGN;
-    if (!aligned(workspace, 256) || workspace_bytes < ca_workspace_bytes(B, H_q, H_kv, C, blk))
+    if (!aligned(workspace, 256) || workspace_bytes < ca::kWorkspaceHeader)
         return CA_ERR_WORKSPACE;
     return CA_OK;
 }
@@ -69,8 +69,16 @@ const char *ca_status_string(int status) {
 int ca_version(void) { return 100; }
 
 size_t ca_workspace_bytes(int B, int H_q, int H_kv, int C, int blk) {
-    if (B <= 0 || H_q <= 0 || H_kv <= 0 || C <= 0 || blk <= 0) return 0;
-    return ca::kWorkspaceHeader;
+    if (B <= 0 || H_q <= 0 || H_kv <= 0 || C <= 0 || blk <= 0 || H_q % H_kv != 0) return 0;
+    // room for the last-wave split of either item layout, at the largest D
+    const int sms = ca::current_sm_count();
+    size_t bytes = ca::kWorkspaceHeader;
+    for (int per_tile = 0; per_tile < 2; ++per_tile) {
+        const int n = ca::attention_items(B, H_q, H_kv, C, per_tile != 0);
+        const ca::SplitPlan plan = ca::plan_split(n, sms, 128, true);
+        if (plan.bytes > bytes) bytes = plan.bytes;
+    }
+    return bytes;
 }
 
 int ca_build_block_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
@@ -97,7 +105,7 @@ int ca_chunk_attention(const void *Q, const void *K, const void *V, const int32_
                                    L_max, D, blk, scale, O, LSE, workspace, workspace_bytes);
     if (st != CA_OK) return st;
     ca::AttnArgs a{Q, K, V, tables, counts, chunk_start, B, H_q, H_kv, C, L_max, D, blk,
-                   scale, O, LSE, workspace};
+                   scale, O, LSE, workspace, workspace_bytes};
     return ca::launch_chunk_attention(a, ca::kModeTables, static_cast<cudaStream_t>(stream));
 }
 
@@ -109,7 +117,7 @@ int ca_dense_chunk_attention(const void *Q, const void *K, const void *V,
                                    L_max, D, blk, scale, O, LSE, workspace, workspace_bytes);
     if (st != CA_OK) return st;
     ca::AttnArgs a{Q, K, V, nullptr, nullptr, chunk_start, B, H_q, H_kv, C, L_max, D, blk,
-                   scale, O, LSE, workspace};
+                   scale, O, LSE, workspace, workspace_bytes};
     return ca::launch_chunk_attention(a, ca::kModeDense, static_cast<cudaStream_t>(stream));
 }
 
@@ -137,7 +145,7 @@ int ca_compacted_chunk_attention(const void *Q, const void *Kc, const void *Vc,
                                    C, L_max, D, blk, scale, O, LSE, workspace, workspace_bytes);
     if (st != CA_OK) return st;
     ca::AttnArgs a{Q, Kc, Vc, tables, counts, chunk_start, B, H_q, H_kv, C, L_max, D, blk,
-                   scale, O, LSE, workspace};
+                   scale, O, LSE, workspace, workspace_bytes};
     return ca::launch_chunk_attention(a, ca::kModeCompact, static_cast<cudaStream_t>(stream));
 }
 
@@ -169,7 +177,7 @@ int ca_tile_chunk_attention(const void *Q, const void *K, const void *V, const i
     if (st != CA_OK) return st;
     if (L_max / blk >= (1 << ca::kSpanEntryBits)) return CA_ERR_SHAPE;
     ca::AttnArgs a{Q, K, V, tables, counts, chunk_start, B, H_q, H_kv, C, L_max, D, blk,
-                   scale, O, LSE, workspace};
+                   scale, O, LSE, workspace, workspace_bytes};
     return ca::launch_chunk_attention(a, ca::kModePerTile, static_cast<cudaStream_t>(stream));
 }
 

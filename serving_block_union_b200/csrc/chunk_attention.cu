@@ -107,6 +107,10 @@ static_assert(kPChunkKeysCfg == 32 || kPChunkKeysCfg == 64 || kPChunkKeysCfg == 
 
 struct Params {
     int B, H_q, H_kv, C, L_max, G, R, n_pairs, nKVmax;
+    int n_items, n_first, split;  // split of the last wave (split == 1: none)
+    unsigned int *counters;       // [n_items - n_first] finished segments per item
+    float *part_lse;              // [n_rest][split][256] base-2 LSE of a segment's rows
+    float *part_o;                // [n_rest][split][256][D] normalised partial O
     float scale_log2;
     const int32_t *tables;
     const int32_t *counts;
@@ -176,6 +180,11 @@ __device__ __forceinline__ constexpr bool use_poly_pair(int q) {
     return kPolyEvery > 0 && (q % kPolyEvery) == kPolyEvery - 1;
 }
 
+// Named barrier 1 over the softmax warps only (barrier 0 is __syncthreads).
+__device__ __forceinline__ void softmax_bar_sync() {
+    asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxWarps * 32) : "memory");
+}
+
 template <int N>
 __device__ __forceinline__ void tmem_ld_row(uint32_t taddr, uint32_t (&r)[N]);
 template <>
@@ -224,16 +233,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *xch_bar = mma_done + 1;  // [2 tiles][4 quarters]: the two half-row warps meet
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xch_bar + 8);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
+    int *last_flag = abort_flag + 1;  // split items: this CTA merges the segments
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     // ---- work item: (b, pair, unit), the unit a KV group, or a query head in
-    // the per-tile mode
+    // the per-tile mode. CTAs [0, n_first) run items [0, n_first) whole; the
+    // rest run one of `split` segments of an item's block list each
+    // (segment-major, so that the CTAs resident together walk the same blocks).
+    int item = blockIdx.x, seg = 0, nseg = 1;
+    if (item >= P.n_first) {
+        const int k = item - P.n_first;
+        const int n_rest = P.n_items - P.n_first;
+        seg = k / n_rest;
+        item = P.n_first + k % n_rest;
+        nseg = P.split;
+    }
     const int units = PERTILE ? P.H_q : P.H_kv;
     const int per_b = units * P.n_pairs;
-    const int b = P.b_order[blockIdx.x / per_b];
-    const int rem = blockIdx.x % per_b;
+    const int b = P.b_order[item / per_b];
+    const int rem = item % per_b;
     const int pair = rem / units;
     const int unit = rem % units;
     const int g = PERTILE ? unit / P.G : unit;     // KV head
@@ -298,6 +318,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         n_eff = count_le<PERTILE>(T, cnt, jlast, lane);
         n_full = count_le<PERTILE>(T, n_eff, jfull, lane);
     }
+    // this CTA's segment of the prefix: table entries [t0, t0 + n_run)
+    const int t0 = (int)((long long)seg * n_eff / nseg);
+    const int n_run = (int)((long long)(seg + 1) * n_eff / nseg) - t0;
 
     // Role code sits inside the branch that re-sized its registers, so the
     // compiler allocates each role within its own budget.
@@ -307,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ================================================================ producer
         int k_issued = 0, v_issued = 0;  // loads started (for the drain below)
         bool q_issued = false;
-        if (n_eff > 0) {
+        if (n_run > 0) {
             if (lane == 0) {
                 mbar_arrive_expect_tx(q_full, 2 * L::kQTile);
                 for (int t = 0; t < 2; ++t)
@@ -318,9 +341,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             q_issued = true;
             int prev_last = -1;
             bool ok = true;
-            for (int w0 = 0; w0 < n_eff && ok; w0 += 32) {
-                const int jj = w0 + lane;
-                const int nwin = min(32, n_eff - w0);
+            for (int w0 = 0; w0 < n_run && ok; w0 += 32) {
+                const int jj = t0 + w0 + lane;  // table index
+                const int nwin = min(32, n_run - w0);
                 int jb = DENSE ? jj : (lane < nwin ? block_of<PERTILE>(__ldg(T + jj)) : 0);
                 if (!DENSE) {
                     int prv = __shfl_up_sync(0xffffffffu, jb, 1);
@@ -335,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 for (int q = 0; q < nwin; ++q) {
                     const int j = w0 + q;
-                    const int blk_idx = COMPACT ? j : __shfl_sync(0xffffffffu, jb, q);
+                    const int blk_idx = COMPACT ? t0 + j : __shfl_sync(0xffffffffu, jb, q);
                     const int s = j % NST;
                     const uint32_t ph = ((j / NST) & 1) ^ 1;
                     int good = 1;
@@ -376,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ================================================================ MMA issue
-        if (n_eff > 0 && lane == 0) {
+        if (n_run > 0 && lane == 0) {
             // Descriptors: the high words are constant; the low words of the Q
             // tiles are fixed for the item and those of a K / V stage are a base
             // plus the stage offset, so each MMA costs one add and the issue.
@@ -427,10 +450,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_commit(s_full + 1);
                 tc_commit(k_empty + 0);
             }
-            for (int j = 0; j < n_eff && ok; ++j) {
+            for (int j = 0; j < n_run && ok; ++j) {
                 const int s = j % NST;
                 const uint32_t ph = (j / NST) & 1;
-                const bool more = j + 1 < n_eff;
+                const bool more = j + 1 < n_run;
                 const int s1 = (j + 1) % NST;
                 const uint32_t ph1 = ((j + 1) / NST) & 1;
                 if (!(ok = mbar_wait(v_full + s, ph, ab))) break;
@@ -503,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         float m_run = -INFINITY, l_run = 0.0f;  // l_run: this warp's columns only
         bool ok = true;
-        for (int j = 0; j < n_eff; ++j) {
+        for (int j = 0; j < n_run; ++j) {
             ok = mbar_wait(s_full + t, j & 1, ab);
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
@@ -511,7 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             int e_j = 0;
-            if (PERTILE) e_j = __ldg(T + j);
+            if (PERTILE) e_j = __ldg(T + t0 + j);
             if (PERTILE && ((e_j >> member_shift) & 1) == 0) {
                 // block not selected by this row's Q-block: P = 0, the running
                 // max and sum are unchanged
@@ -538,8 +561,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < CW; ++i) s[i] = __uint_as_float(v[i]);
             }
-            if (j >= n_full) {
-                int jb = DENSE ? j : (PERTILE ? block_of<true>(e_j) : __ldg(T + j));
+            if (t0 + j >= n_full) {
+                int jb = DENSE ? t0 + j : (PERTILE ? block_of<true>(e_j) : __ldg(T + t0 + j));
                 jb = min(max(jb, 0), P.nKVmax);  // only matters for a flagged, invalid table
                 const int lim = p - jb * BLK - hf * CW;  // columns c <= lim are visible
 #pragma unroll
@@ -631,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             l_run += sum;
         }
         bool have_o = false;
-        if (n_eff > 0 && __all_sync(0xffffffffu, ok)) {
+        if (n_run > 0 && __all_sync(0xffffffffu, ok)) {
             const bool got = mbar_wait(o_full + t, 0, ab);
             have_o = __all_sync(0xffffffffu, got);
             tc_fence_after();
@@ -645,31 +668,115 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+        const float lse2 = (l_run > 0.0f && have_o) ? m_run + log2f(l_run) : -INFINITY;
         uint16_t *orow = P.O + (((size_t)b * P.H_q + h) * P.C + r) * D + hf * DW;
+        float *lse_out = (valid && hf == 0 && P.LSE != nullptr)
+                             ? P.LSE + ((size_t)b * P.H_q + h) * P.C + r
+                             : nullptr;
+        if (nseg == 1) {
 #pragma unroll
-        for (int c = 0; c < DW / 32; ++c) {
-            uint32_t v[32];
-            if (have_o) {
-                tmem_ld32(tO + c * 32, v);
-            } else {
+            for (int c = 0; c < DW / 32; ++c) {
+                uint32_t v[32];
+                if (have_o) {
+                    tmem_ld32(tO + c * 32, v);
+                } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = 0u;
+                    for (int i = 0; i < 32; ++i) v[i] = 0u;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l,
+                                        __uint_as_float(v[2 * i + 1]) * inv_l);
+                if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                }
             }
-            uint32_t pk[16];
+            if (lse_out) *lse_out = lse2 * kLn2;
+        } else {
+            // Segment of a split item: its normalised O (fp32) and base-2 LSE
+            // go to the workspace, one slot row per packed row.
+            const int rest = item - P.n_first;
+            const size_t row0 = (size_t)rest * nseg * kRowsPerItem + t * 128 + m;
+            const size_t mine = row0 + (size_t)seg * kRowsPerItem;
+            float *po = P.part_o + mine * D + hf * DW;
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l,
-                                    __uint_as_float(v[2 * i + 1]) * inv_l);
-            if (valid) {
-                uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+            for (int c = 0; c < DW / 32; ++c) {
+                uint32_t v[32];
+                if (have_o) {
+                    tmem_ld32(tO + c * 32, v);
+                } else {
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    for (int i = 0; i < 32; ++i) v[i] = 0u;
+                }
+                float4 *dst = reinterpret_cast<float4 *>(po + c * 32);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dst[i] = make_float4(__uint_as_float(v[4 * i]) * inv_l,
+                                         __uint_as_float(v[4 * i + 1]) * inv_l,
+                                         __uint_as_float(v[4 * i + 2]) * inv_l,
+                                         __uint_as_float(v[4 * i + 3]) * inv_l);
             }
-        }
-        if (valid && hf == 0 && P.LSE != nullptr) {
-            P.LSE[((size_t)b * P.H_q + h) * P.C + r] =
-                (l_run > 0.0f && have_o) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+            if (hf == 0) P.part_lse[mine] = lse2;
+            // publish, count this segment in, and let the item's last CTA merge
+            __threadfence();
+            softmax_bar_sync();
+            if (threadIdx.x == 0) {
+                const unsigned prev = atomicAdd(P.counters + rest, 1u);
+                *last_flag = prev + 1 == (unsigned)nseg;
+            }
+            softmax_bar_sync();
+            if (*last_flag) {
+                __threadfence();
+                float ls[kMaxSplit];
+                float mx = -INFINITY;
+#pragma unroll
+                for (int sg = 0; sg < kMaxSplit; ++sg) {
+                    ls[sg] = sg < nseg ? __ldcg(P.part_lse + row0 + (size_t)sg * kRowsPerItem)
+                                       : -INFINITY;
+                    mx = fmaxf(mx, ls[sg]);
+                }
+                float wsum = 0.0f;
+#pragma unroll
+                for (int sg = 0; sg < kMaxSplit; ++sg) {
+                    ls[sg] = mx == -INFINITY ? 0.0f : exp2f(ls[sg] - mx);  // weight
+                    wsum += ls[sg];
+                }
+                const float inv_w = wsum > 0.0f ? 1.0f / wsum : 0.0f;
+#pragma unroll
+                for (int c = 0; c < DW / 32; ++c) {
+                    float acc[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
+                    for (int sg = 0; sg < nseg; ++sg) {
+                        const float w = ls[sg] * inv_w;
+                        const float4 *src = reinterpret_cast<const float4 *>(
+                            P.part_o + (row0 + (size_t)sg * kRowsPerItem) * D + hf * DW + c * 32);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float4 x = __ldcg(src + i);
+                            acc[4 * i] = fmaf(w, x.x, acc[4 * i]);
+                            acc[4 * i + 1] = fmaf(w, x.y, acc[4 * i + 1]);
+                            acc[4 * i + 2] = fmaf(w, x.z, acc[4 * i + 2]);
+                            acc[4 * i + 3] = fmaf(w, x.w, acc[4 * i + 3]);
+                        }
+                    }
+                    if (valid) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(pack_bf16x2(acc[8 * i], acc[8 * i + 1]),
+                                                pack_bf16x2(acc[8 * i + 2], acc[8 * i + 3]),
+                                                pack_bf16x2(acc[8 * i + 4], acc[8 * i + 5]),
+                                                pack_bf16x2(acc[8 * i + 6], acc[8 * i + 7]));
+                    }
+                }
+                if (lse_out) *lse_out = wsum > 0.0f ? (mx + log2f(wsum)) * kLn2 : -INFINITY;
+                if (threadIdx.x == 0) P.counters[rest] = 0u;  // ready for the next launch
+            }
         }
     }
 
@@ -777,13 +884,49 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
         P.chunk_start[i] = i < a.B ? a.chunk_start[i] : 0;
         P.b_order[i] = static_cast<unsigned char>(i < a.B ? order[i] : 0);
     }
+    // split the last wave when the items are alike (one cache length) and long
     const int units = MODE == kModePerTile ? a.H_q : a.H_kv;
-    const unsigned grid = static_cast<unsigned>(a.B * units * n_pairs);
+    const int n_items = a.B * units * n_pairs;
+    bool alike = true;
+    int nkv_max = 0;
+    for (int i = 0; i < a.B; ++i) {
+        alike = alike && a.chunk_start[i] == a.chunk_start[0];
+        nkv_max = max(nkv_max, (a.chunk_start[i] + a.C + BLK - 1) / BLK);
+    }
+    SplitPlan plan = plan_split(n_items, current_sm_count(), D,
+                                alike && nkv_max >= kSplitMinBlocks);
+    if (plan.split > 1 && a.workspace_bytes < plan.bytes)
+        plan = plan_split(n_items, 0, D, false);  // workspace too small: no split
+    unsigned char *ws = static_cast<unsigned char *>(a.workspace);
+    P.n_items = n_items;
+    P.n_first = plan.n_first;
+    P.split = plan.split;
+    P.counters = reinterpret_cast<unsigned int *>(ws + kWorkspaceHeader);
+    P.part_lse = reinterpret_cast<float *>(ws + plan.lse_off);
+    P.part_o = reinterpret_cast<float *>(ws + plan.o_off);
+    const unsigned grid = static_cast<unsigned>(plan.n_first +
+                                                (n_items - plan.n_first) * plan.split);
     kern<<<grid, kThreads, L::kDynamic, stream>>>(tq, tk, tv, P);
     return cudaGetLastError() == cudaSuccess ? CA_OK : CA_ERR_CUDA;
 }
 
 }  // namespace
+
+int current_sm_count() {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            n <= 0)
+            return 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
 
 int launch_chunk_attention(const AttnArgs &a, int mode, cudaStream_t stream) {
 #define CA_DISPATCH(D_, BLK_)                                                         \

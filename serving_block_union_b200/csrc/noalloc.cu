@@ -22,10 +22,12 @@
 
 namespace {
 
-// Largest workspace this entry point can provide. ca_workspace_bytes is a
-// constant 256 bytes for the current kernels (the device status word and
-// scheduler header); calls that would need more are rejected.
+// Size of the library's scratch array. The attention kernels need a 256-byte
+// header (the device status word) at minimum; the partial results of the
+// last-wave split need far more, so the kernels, seeing a workspace this
+// small, run unsplit.
 constexpr size_t kNoAllocScratchBytes = 4096;
+static_assert(kNoAllocScratchBytes >= ca::kWorkspaceHeader, "scratch below the minimum");
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char ca_noalloc_scratch[kNoAllocScratchBytes];
@@ -55,9 +57,7 @@ extern "C" int ca_chunk_attention_noalloc(const void *Q, const void *K, const vo
                                           const int32_t *chunk_start, int B, int H_q, int H_kv,
                                           int C, int L_max, int D, int blk, float scale, void *O,
                                           float *LSE, unsigned int *device_status, void *stream) {
-    const size_t need = ca_workspace_bytes(B, H_q, H_kv, C, blk);
-    if (need == 0) return CA_ERR_INVALID_ARG;
-    if (need > kNoAllocScratchBytes) return CA_ERR_WORKSPACE;
+    if (ca_workspace_bytes(B, H_q, H_kv, C, blk) == 0) return CA_ERR_INVALID_ARG;
     void *scratch = nullptr;
     const int st = scratch_for_current_device(&scratch);
     if (st != CA_OK) return st;

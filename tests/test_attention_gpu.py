@@ -115,6 +115,54 @@ def test_tiny_workload_tables_from_gpu_builder(cuda_ok):
     compare(O, L, O_ref, L_ref)
 
 
+# ------------------------------------------------------- split of the last wave
+
+SPLIT = [
+    # B, H_q, H_kv, D, blk, C, L_max, chunk_start: few items over long caches,
+    # so the launch cuts every item into segments merged through the workspace
+    (1, 4, 1, 128, 64, 256, 64 * 80, (64 * 76,)),        # 4 items -> 8 segments each
+    (2, 8, 2, 64, 128, 384, 128 * 72, (128 * 64, 128 * 64)),
+    (1, 32, 8, 128, 128, 128, 128 * 70, (128 * 69,)),    # G = 4, 16 items
+]
+
+
+@pytest.mark.parametrize("case", SPLIT)
+def test_split_last_wave_full_compare(cuda_ok, case):
+    B, H_q, H_kv, D, blk, C, L_max, cs = case
+    mask, Q, K, V = _small_case(B, H_q, H_kv, D, blk, C, L_max, cs, 0.3, seed=sum(case[:7]))
+    T, c, _, _ = oracle.block_tables(mask, H_q // H_kv)
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    Td, cd = torch.from_numpy(T).cuda(), torch.from_numpy(c).cuda()
+    ws = ca.new_workspace(B, H_q, H_kv, C, blk)
+    assert ws.numel() > 256  # room for the split on this device
+    O, L = ca.chunk_attention(Qd, Kd, Vd, Td, cd, cs, workspace=ws)
+    assert ca.read_device_status(ws) == ca.CA_OK
+    # every merge counter (one uint32 per split item, after the 256-byte
+    # header) is back at zero, ready for the next call
+    G = H_q // H_kv
+    items = B * H_kv * ((-(-C // (128 // G)) + 1) // 2)
+    assert items < 148
+    assert int(ws[256:256 + 4 * items].count_nonzero()) == 0
+    O_ref, L_ref = oracle.attention(Q, K, V, cs, blk, T, c)
+    compare(O, L, O_ref, L_ref)
+    # the same call on a minimal workspace runs unsplit: same result within rounding
+    ws_min = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    O1, L1 = ca.chunk_attention(Qd, Kd, Vd, Td, cd, cs, workspace=ws_min)
+    compare(O1, L1, O_ref, L_ref)
+    # reusing the workspace gives the identical result
+    O2, L2 = ca.chunk_attention(Qd, Kd, Vd, Td, cd, cs, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(O, O2) and torch.equal(L, L2)
+
+
+def test_split_dense_full_compare(cuda_ok):
+    B, H_q, H_kv, D, blk, C, L_max, cs = SPLIT[0]
+    _, Q, K, V = _small_case(B, H_q, H_kv, D, blk, C, L_max, cs, 0.0, seed=31)
+    O, L = _run_gpu(Q, K, V, None, None, cs, dense=True, blk=blk)
+    O_ref, L_ref = oracle.attention(Q, K, V, cs, blk)
+    compare(O, L, O_ref, L_ref)
+
+
 # ------------------------------------------------------------------ full sizes
 
 FULL = ["llama8b_32k", "llama8b_128k_d2", "llama8b_128k_d5", "llama8b_128k_d10",

@@ -65,6 +65,20 @@ def test_small_shapes_tables_and_attention(cuda_ok, case, p):
     compare(O, L, O_ref, L_ref)
 
 
+def test_split_last_wave(cuda_ok):
+    """Few per-head items over a long cache: segments merged through the
+    workspace, checked against the oracle in full."""
+    B, H_q, H_kv, D, blk, C, L_max, cs = 1, 4, 2, 128, 128, 512, 128 * 80, (128 * 76,)
+    mask, Q, K, V = _small_case(B, H_q, H_kv, D, blk, C, L_max, 0.3, seed=41)
+    ws = ca.new_workspace(B, H_q, H_kv, C, blk)
+    _, _, O, L = _gpu_tile(mask, Q, K, V, cs, blk, ws=ws)
+    assert ca.read_device_status(ws) == ca.CA_OK
+    items = B * H_q * (-(-C // 256))  # per-head items, one merge counter each
+    assert int(ws[256:256 + 4 * items].count_nonzero()) == 0
+    O_ref, L_ref = oracle.attention_tile(Q, K, V, cs, blk, mask)
+    compare(O, L, O_ref, L_ref)
+
+
 def test_rows_without_keys(cuda_ok):
     """A Q-block that selects nothing (or only future blocks) gives O = 0 and
     LSE = -inf on its rows, whatever its span partner selects."""
