@@ -128,6 +128,42 @@ int ca_chunk_attention(const void *Q, const void *K, const void *V, const int32_
                        float *LSE, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Block-Union tables in the paged-kernel metadata form (pages: "Methodology",
+ * execution stage — the tables reach the paged attention kernel as
+ * kv_indptr / kv_indices). Same union as ca_build_block_tables (tables and
+ * counts are written too), and
+ *   kv_indptr[k]  = sum of counts over flattened (b, g) < k   (k = 0..B*H_kv)
+ *   kv_indices[kv_indptr[b*H_kv+g] + t] = (b*H_kv + g) * nKVmax + T_{b,g}[t]
+ * i.e. global page ids of the cache viewed as B*H_kv*nKVmax pages of blk rows.
+ * kv_indptr int32 [B*H_kv + 1], kv_indices int32 [B*H_kv*nKVmax] (capacity;
+ * the first kv_indptr[B*H_kv] entries are written). Errors as
+ * ca_build_block_tables; both pointers are required.
+ */
+int ca_build_kv_pages(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
+                      int32_t *tables, int32_t *counts, int32_t *kv_indptr, int32_t *kv_indices,
+                      void *stream);
+
+/*
+ * ca_chunk_attention over the paged metadata form, with chunks of different
+ * lengths (ragged batches): the block list of (b, g) is
+ *   { kv_indices[t] - (b*H_kv + g) * nKVmax : kv_indptr[b*H_kv+g] <= t < kv_indptr[b*H_kv+g+1] },
+ * ascending, and sequence b has chunk_len[b] rows (0 <= chunk_len[b] <= C;
+ * NULL = all C). Q / O stay padded [B, H_q, C, D] (LSE [B, H_q, C]); rows
+ * r >= chunk_len[b] are neither read for their result nor written. Each row's
+ * result is the one ca_chunk_attention defines, with
+ * chunk_start[b] + chunk_len[b] <= L_max instead of chunk_start[b] + C.
+ * kv_indptr int32 [B*H_kv + 1] and kv_indices int32 [nnz] are device arrays.
+ * A row range outside [0, nnz], longer than nKVmax or decreasing, or an entry
+ * that is not a page of its own (b, g), is a device error (CA_ERR_TABLE) that
+ * skips the affected work. Other arguments and errors as ca_chunk_attention.
+ */
+int ca_paged_chunk_attention(const void *Q, const void *K, const void *V,
+                             const int32_t *kv_indptr, const int32_t *kv_indices, long long nnz,
+                             const int32_t *chunk_start, const int32_t *chunk_len, int B, int H_q,
+                             int H_kv, int C, int L_max, int D, int blk, float scale, void *O,
+                             float *LSE, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * The dense paged path (pages: the "dense attention baseline" the speedup is
  * quoted against): identical to ca_chunk_attention with
  * T_{b,g} = [0, ceil((chunk_start[b] + C) / blk)) for every group.

@@ -70,6 +70,8 @@ EXPORTED_SYMBOLS = (
     "ca_compact_kv_blocks",
     "ca_compacted_chunk_attention",
     "ca_tile_span",
+    "ca_build_kv_pages",
+    "ca_paged_chunk_attention",
     "ca_build_tile_tables",
     "ca_tile_chunk_attention",
 )
@@ -120,6 +122,11 @@ def load_library():
         lib.ca_compacted_chunk_attention.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P,
                                                      P, P, S, P]
         lib.ca_compacted_chunk_attention.restype = I
+        lib.ca_build_kv_pages.argtypes = [P, I, I, I, I, I, P, P, P, P, P]
+        lib.ca_build_kv_pages.restype = I
+        lib.ca_paged_chunk_attention.argtypes = [P, P, P, P, P, ctypes.c_longlong, P, P, I, I, I,
+                                                 I, I, I, I, F, P, P, P, S, P]
+        lib.ca_paged_chunk_attention.restype = I
         lib.ca_tile_span.argtypes = [I]
         lib.ca_tile_span.restype = I
         lib.ca_build_tile_tables.argtypes = [P, I, I, I, I, I, P, P, P]
@@ -209,6 +216,30 @@ def build_block_tables(mask: torch.Tensor, group: int, csr: bool = False,
                                    _stream_handle(stream, dev))
     _check("ca_build_block_tables", st)
     return tables, counts, indptr, indices
+
+
+def build_kv_pages(mask: torch.Tensor, group: int, stream: Optional[torch.cuda.Stream] = None):
+    """Block-Union tables in the paged metadata form: ``(kv_indptr int32
+    [B*H_kv+1], kv_indices int32 [B*H_kv*nKVmax])`` with global page ids
+    ``(b*H_kv + g)*nKVmax + j``; the valid part of ``kv_indices`` is
+    ``kv_indices[:kv_indptr[-1]]``. Also returns the dense ``tables, counts``."""
+    if mask.dtype == torch.bool:
+        mask = mask.view(torch.uint8)
+    _need(mask, "mask", torch.uint8, 4)
+    B, H_q, nQ, nK = mask.shape
+    if group <= 0 or H_q % group:
+        raise ValueError("group must divide H_q")
+    H_kv = H_q // group
+    dev = mask.device
+    tables = torch.empty((B, H_kv, nK), dtype=torch.int32, device=dev)
+    counts = torch.empty((B, H_kv), dtype=torch.int32, device=dev)
+    indptr = torch.empty(B * H_kv + 1, dtype=torch.int32, device=dev)
+    indices = torch.empty(B * H_kv * nK, dtype=torch.int32, device=dev)
+    st = load_library().ca_build_kv_pages(_ptr(mask), B, H_q, nQ, nK, int(group), _ptr(tables),
+                                          _ptr(counts), _ptr(indptr), _ptr(indices),
+                                          _stream_handle(stream, dev))
+    _check("ca_build_kv_pages", st)
+    return indptr, indices, tables, counts
 
 
 # ----------------------------------------------------------------- attention
@@ -482,4 +513,35 @@ def tile_chunk_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, tabl
         blk, float(scale), _ptr(O), _ptr(LSE), _ptr(workspace), workspace.numel(),
         _stream_handle(stream, Q.device))
     _check("ca_tile_chunk_attention", st)
+    return O, LSE
+
+
+# -------------------------------------------- paged metadata, ragged chunks
+
+def paged_chunk_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                          kv_indptr: torch.Tensor, kv_indices: torch.Tensor,
+                          chunk_start: Sequence[int], blk: int,
+                          chunk_len: Optional[Sequence[int]] = None,
+                          scale: Optional[float] = None, O: Optional[torch.Tensor] = None,
+                          LSE: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None,
+                          stream: Optional[torch.cuda.Stream] = None
+                          ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """chunk_attention over the ``kv_indptr`` / ``kv_indices`` (global page)
+    form, with per-sequence chunk lengths ``chunk_len`` (rows past a
+    sequence's length are left untouched in ``O`` / ``LSE``)."""
+    _need(kv_indptr, "kv_indptr", torch.int32, 1)
+    _need(kv_indices, "kv_indices", torch.int32, 1)
+    B, H_q, H_kv, C, L_max, D, O, LSE, workspace = _attn_common(Q, K, V, O, LSE, workspace, blk)
+    if kv_indptr.numel() != B * H_kv + 1:
+        raise ValueError("kv_indptr must have B*H_kv + 1 entries")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    cs = _chunk_start_host(chunk_start, B)
+    cl = None if chunk_len is None else _chunk_start_host(chunk_len, B)
+    st = load_library().ca_paged_chunk_attention(
+        _ptr(Q), _ptr(K), _ptr(V), _ptr(kv_indptr), _ptr(kv_indices), kv_indices.numel(), cs, cl,
+        B, H_q, H_kv, C, L_max, D, int(blk), float(scale), _ptr(O), _ptr(LSE), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream, Q.device))
+    _check("ca_paged_chunk_attention", st)
     return O, LSE

@@ -140,7 +140,8 @@ __global__ void __launch_bounds__(kMaxThreads)
 // CSR form: indptr[bg] = sum of counts before bg; indices = valid prefixes.
 __global__ void __launch_bounds__(256)
     csr_kernel(const int32_t *__restrict__ tables, const int32_t *__restrict__ counts, int n_bg,
-               int nKVmax, int32_t *__restrict__ indptr, int32_t *__restrict__ indices) {
+               int nKVmax, bool page_ids, int32_t *__restrict__ indptr,
+               int32_t *__restrict__ indices) {
     __shared__ int red[256];
     const int bg = blockIdx.x, tid = threadIdx.x;
     int s = 0;
@@ -158,8 +159,10 @@ __global__ void __launch_bounds__(256)
         if (bg == n_bg - 1) indptr[n_bg] = off + n;
     }
     if (indices) {
+        // block j of (b, g), or its global page (b * H_kv + g) * nKVmax + j
         const int32_t *T = tables + (size_t)bg * nKVmax;
-        for (int t = tid; t < n; t += blockDim.x) indices[off + t] = T[t];
+        const int32_t base = page_ids ? bg * nKVmax : 0;
+        for (int t = tid; t < n; t += blockDim.x) indices[off + t] = base + T[t];
     }
 }
 
@@ -167,7 +170,7 @@ __global__ void __launch_bounds__(256)
 
 int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
                         int32_t *tables, int32_t *counts, int32_t *indptr, int32_t *indices,
-                        cudaStream_t stream) {
+                        bool page_ids, cudaStream_t stream) {
     const int H_kv = H_q / group;
     const int n_chunks = (nKVmax + 15) / 16;
     int chp = ((n_chunks + 31) / 32) * 32;
@@ -186,8 +189,8 @@ int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax,
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return CA_ERR_CUDA;
     if (indptr) {
-        csr_kernel<<<B * H_kv, 256, 0, stream>>>(tables, counts, B * H_kv, nKVmax, indptr,
-                                                  indices);
+        csr_kernel<<<B * H_kv, 256, 0, stream>>>(tables, counts, B * H_kv, nKVmax, page_ids,
+                                                  indptr, indices);
         e = cudaGetLastError();
         if (e != cudaSuccess) return CA_ERR_CUDA;
     }

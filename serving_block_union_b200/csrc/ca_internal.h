@@ -16,9 +16,10 @@ constexpr int kMaxBatch = 128;
 // [8, 12) finished-CTA counter; padded to 256.
 constexpr size_t kWorkspaceHeader = 256;
 
+// page_ids: CSR indices hold global pages (b * H_kv + g) * nKVmax + j.
 int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
                         int32_t *tables, int32_t *counts, int32_t *indptr, int32_t *indices,
-                        cudaStream_t stream);
+                        bool page_ids, cudaStream_t stream);
 
 struct AttnArgs {
     const void *Q, *K, *V;
@@ -30,6 +31,11 @@ struct AttnArgs {
     float *LSE;
     void *workspace;
     size_t workspace_bytes;
+    // paged form (kModeTables only): tables = kv_indices (global pages, nnz
+    // entries), counts unused, rows of (b, g) at kv_indptr[b*H_kv+g] ..
+    const int32_t *kv_indptr = nullptr;
+    long long nnz = 0;
+    const int32_t *chunk_len = nullptr;  // host [B], NULL: every chunk is C rows
 };
 
 // Attention kernel modes: walk the tables over the cache in place; every block

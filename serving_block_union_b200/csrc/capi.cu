@@ -19,7 +19,8 @@ inline bool supported_group(int G) { return G == 1 || G == 2 || G == 4 || G == 8
 int check_attention(const void *Q, const void *K, const void *V, const int32_t *tables,
                     const int32_t *counts, bool dense, const int32_t *chunk_start, int B, int H_q,
                     int H_kv, int C, int L_max, int D, int blk, float scale, const void *O,
-                    const float *LSE, const void *workspace, size_t workspace_bytes) {
+                    const float *LSE, const void *workspace, size_t workspace_bytes,
+                    const int32_t *chunk_len = nullptr) {
     if (!Q || !K || !V || !O || !chunk_start || !workspace) return CA_ERR_INVALID_ARG;
     if (!dense && (!tables || !counts)) return CA_ERR_INVALID_ARG;
     if (B <= 0 || H_q <= 0 || H_kv <= 0 || C <= 0 || L_max <= 0 || D <= 0 || blk <= 0)
@@ -29,7 +30,9 @@ int check_attention(const void *Q, const void *K, const void *V, const int32_t *
     if (L_max % blk != 0) return CA_ERR_SHAPE;
     for (int b = 0; b < B && b < ca::kMaxBatch; ++b) {
         const long long cs = chunk_start[b];
-        if (cs < 0 || cs + C > L_max) return CA_ERR_SHAPE;
+        const long long len = chunk_len ? chunk_len[b] : C;
+        if (len < 0 || len > C) return CA_ERR_SHAPE;
+        if (cs < 0 || cs + len > L_max) return CA_ERR_SHAPE;
     }
     if (!(D == 64 || D == 128) || !(blk == 64 || blk == 128)) return CA_ERR_UNSUPPORTED;
     if (!supported_group(H_q / H_kv)) return CA_ERR_UNSUPPORTED;
@@ -94,7 +97,41 @@ int ca_build_block_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVma
         (indices && !aligned(indices, 4)))
         return CA_ERR_ALIGN;
     return ca::launch_build_tables(mask, B, H_q, nQ, nKVmax, group, tables, counts, indptr,
-                                   indices, static_cast<cudaStream_t>(stream));
+                                   indices, false, static_cast<cudaStream_t>(stream));
+}
+
+int ca_build_kv_pages(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
+                      int32_t *tables, int32_t *counts, int32_t *kv_indptr, int32_t *kv_indices,
+                      void *stream) {
+    if (!kv_indptr || !kv_indices) return CA_ERR_INVALID_ARG;
+    if (!mask || !tables || !counts) return CA_ERR_INVALID_ARG;
+    if (B <= 0 || H_q <= 0 || nQ <= 0 || nKVmax <= 0 || group <= 0) return CA_ERR_INVALID_ARG;
+    if (H_q % group != 0) return CA_ERR_SHAPE;
+    if ((long long)B * H_q * nQ * nKVmax >= (1LL << 40)) return CA_ERR_SHAPE;
+    if ((long long)B * (H_q / group) * nKVmax >= (1LL << 31)) return CA_ERR_SHAPE;
+    if (!aligned(tables, 4) || !aligned(counts, 4) || !aligned(kv_indptr, 4) ||
+        !aligned(kv_indices, 4))
+        return CA_ERR_ALIGN;
+    return ca::launch_build_tables(mask, B, H_q, nQ, nKVmax, group, tables, counts, kv_indptr,
+                                   kv_indices, true, static_cast<cudaStream_t>(stream));
+}
+
+int ca_paged_chunk_attention(const void *Q, const void *K, const void *V,
+                             const int32_t *kv_indptr, const int32_t *kv_indices, long long nnz,
+                             const int32_t *chunk_start, const int32_t *chunk_len, int B, int H_q,
+                             int H_kv, int C, int L_max, int D, int blk, float scale, void *O,
+                             float *LSE, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!kv_indptr || !kv_indices || nnz < 0) return CA_ERR_INVALID_ARG;
+    const int st = check_attention(Q, K, V, kv_indices, kv_indptr, false, chunk_start, B, H_q,
+                                   H_kv, C, L_max, D, blk, scale, O, LSE, workspace,
+                                   workspace_bytes, chunk_len);
+    if (st != CA_OK) return st;
+    ca::AttnArgs a{Q, K, V, kv_indices, nullptr, chunk_start, B, H_q, H_kv, C, L_max, D, blk,
+                   scale, O, LSE, workspace, workspace_bytes};
+    a.kv_indptr = kv_indptr;
+    a.nnz = nnz;
+    a.chunk_len = chunk_len;
+    return ca::launch_chunk_attention(a, ca::kModeTables, static_cast<cudaStream_t>(stream));
 }
 
 int ca_chunk_attention(const void *Q, const void *K, const void *V, const int32_t *tables,

@@ -112,12 +112,15 @@ struct Params {
     float *part_lse;              // [n_rest][split][256] base-2 LSE of a segment's rows
     float *part_o;                // [n_rest][split][256][D] normalised partial O
     float scale_log2;
-    const int32_t *tables;
+    const int32_t *tables;      // or, in the paged form, kv_indices (global pages)
     const int32_t *counts;
+    const int32_t *kv_indptr;   // paged form: rows of (b, g) in kv_indices; else NULL
+    long long nnz;              // paged form: entries of kv_indices
     uint16_t *O;
     float *LSE;
     unsigned int *status;
     int chunk_start[kMaxBatch];
+    int chunk_len[kMaxBatch];   // rows of each sequence's chunk (<= C)
     unsigned char b_order[kMaxBatch];
 };
 
@@ -153,12 +156,12 @@ __device__ __forceinline__ int block_of(int e) {
 // (all 32 lanes), scanning windows of 32 from the end (the answer is normally
 // in the last window: only blocks inside the chunk can lie past the bound).
 template <bool SPAN>
-__device__ __forceinline__ int count_le(const int32_t *T, int n, int bound, int lane) {
+__device__ __forceinline__ int count_le(const int32_t *T, int n, int bound, int lane, int base) {
     int hi = n;
     while (hi > 0) {
         const int lo = hi > 32 ? hi - 32 : 0;
         const int idx = lo + lane;
-        const int v = idx < hi ? block_of<SPAN>(__ldg(T + idx)) : 0;
+        const int v = idx < hi ? block_of<SPAN>(__ldg(T + idx)) - base : 0;
         const unsigned gt = __ballot_sync(0xffffffffu, idx < hi && v > bound);
         const int ngt = __popc(gt);
         if (ngt < hi - lo) return hi - ngt;
@@ -259,9 +262,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = PERTILE ? unit / P.G : unit;     // KV head
     const int head0 = PERTILE ? unit : g * P.G;  // query head of packed row 0
     const int cs = P.chunk_start[b];
+    const int len_b = P.chunk_len[b];  // this sequence's chunk rows
     const int R = P.R;
     const int r0 = pair * 2 * R;
-    const int r_end = min(r0 + 2 * R, P.C);
+    const int r_end = min(r0 + 2 * R, len_b);
     const int p_min = cs + r0;
     const int p_max = cs + r_end - 1;
     const int jlast = p_max / BLK;
@@ -302,21 +306,37 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- table prefix this item walks (every role computes it the same way)
     const int32_t *T = nullptr;
+    int base = 0;  // paged form: entries are base + block index
     int n_eff, n_full;
-    if (DENSE) {
+    if (r0 >= len_b) {  // a pair past a shorter chunk's end: no rows, no work
+        n_eff = n_full = 0;
+    } else if (DENSE) {
         n_eff = jlast + 1;
         n_full = jfull + 1 > 0 ? jfull + 1 : 0;
     } else {
         const size_t trow = PERTILE ? ((size_t)b * P.H_q + unit) * P.n_pairs + pair
                                     : (size_t)b * P.H_kv + g;
-        int cnt = __ldg(P.counts + trow);
-        if (cnt < 0 || cnt > P.nKVmax) {
-            if (threadIdx.x == 0) atomicOr(P.status, kDevErrTable);
-            cnt = 0;
+        int cnt;
+        if (!PERTILE && P.kv_indptr != nullptr) {
+            const long long start = __ldg(P.kv_indptr + trow);
+            const long long end = __ldg(P.kv_indptr + trow + 1);
+            cnt = (int)(end - start);
+            if (start < 0 || end > P.nnz || end < start || end - start > P.nKVmax) {
+                if (threadIdx.x == 0) atomicOr(P.status, kDevErrTable);
+                cnt = 0;
+            }
+            T = P.tables + (cnt > 0 ? start : 0);
+            base = (int)trow * P.nKVmax;
+        } else {
+            cnt = __ldg(P.counts + trow);
+            if (cnt < 0 || cnt > P.nKVmax) {
+                if (threadIdx.x == 0) atomicOr(P.status, kDevErrTable);
+                cnt = 0;
+            }
+            T = P.tables + trow * P.nKVmax;
         }
-        T = P.tables + trow * P.nKVmax;
-        n_eff = count_le<PERTILE>(T, cnt, jlast, lane);
-        n_full = count_le<PERTILE>(T, n_eff, jfull, lane);
+        n_eff = count_le<PERTILE>(T, cnt, jlast, lane, base);
+        n_full = count_le<PERTILE>(T, n_eff, jfull, lane, base);
     }
     // this CTA's segment of the prefix: table entries [t0, t0 + n_run)
     const int t0 = (int)((long long)seg * n_eff / nseg);
@@ -344,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int w0 = 0; w0 < n_run && ok; w0 += 32) {
                 const int jj = t0 + w0 + lane;  // table index
                 const int nwin = min(32, n_run - w0);
-                int jb = DENSE ? jj : (lane < nwin ? block_of<PERTILE>(__ldg(T + jj)) : 0);
+                int jb = DENSE ? jj : (lane < nwin ? block_of<PERTILE>(__ldg(T + jj)) - base : 0);
                 if (!DENSE) {
                     int prv = __shfl_up_sync(0xffffffffu, jb, 1);
                     if (lane == 0) prv = prev_last;
@@ -496,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int m = qw * 32 + lane;
         const int h_local = m / R;
         const int r = r0 + t * R + (m % R);
-        const bool valid = r < P.C;
+        const bool valid = r < len_b;
         const int p = cs + r;
         const int h = head0 + h_local;
         // per-tile mode: bit of this row's Q-block in the span-table entries
@@ -562,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < CW; ++i) s[i] = __uint_as_float(v[i]);
             }
             if (t0 + j >= n_full) {
-                int jb = DENSE ? t0 + j : (PERTILE ? block_of<true>(e_j) : __ldg(T + t0 + j));
+                int jb = DENSE ? t0 + j : (PERTILE ? block_of<true>(e_j) : __ldg(T + t0 + j) - base);
                 jb = min(max(jb, 0), P.nKVmax);  // only matters for a flagged, invalid table
                 const int lim = p - jb * BLK - hf * CW;  // columns c <= lim are visible
 #pragma unroll
@@ -865,16 +885,20 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
     P.scale_log2 = a.scale * 1.4426950408889634f;
     P.tables = a.tables;
     P.counts = a.counts;
+    P.kv_indptr = a.kv_indptr;
+    P.nnz = a.nnz;
     P.O = static_cast<uint16_t *>(a.O);
     P.LSE = a.LSE;
     P.status = static_cast<unsigned int *>(a.workspace);
-    // longest sequences first: their items are the heaviest
+    // longest visible lengths first: their items are the heaviest
+    auto len_of = [&](int i) { return a.chunk_len ? a.chunk_len[i] : a.C; };
+    auto reach = [&](int i) { return (long long)a.chunk_start[i] + len_of(i); };
     int order[kMaxBatch];
     for (int i = 0; i < a.B; ++i) order[i] = i;
     for (int i = 1; i < a.B; ++i) {
         const int x = order[i];
         int k = i - 1;
-        while (k >= 0 && a.chunk_start[order[k]] < a.chunk_start[x]) {
+        while (k >= 0 && reach(order[k]) < reach(x)) {
             order[k + 1] = order[k];
             --k;
         }
@@ -882,6 +906,7 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
     }
     for (int i = 0; i < kMaxBatch; ++i) {
         P.chunk_start[i] = i < a.B ? a.chunk_start[i] : 0;
+        P.chunk_len[i] = i < a.B ? len_of(i) : 0;
         P.b_order[i] = static_cast<unsigned char>(i < a.B ? order[i] : 0);
     }
     // split the last wave when the items are alike (one cache length) and long
@@ -890,8 +915,8 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
     bool alike = true;
     int nkv_max = 0;
     for (int i = 0; i < a.B; ++i) {
-        alike = alike && a.chunk_start[i] == a.chunk_start[0];
-        nkv_max = max(nkv_max, (a.chunk_start[i] + a.C + BLK - 1) / BLK);
+        alike = alike && a.chunk_start[i] == a.chunk_start[0] && len_of(i) == len_of(0);
+        nkv_max = max(nkv_max, (a.chunk_start[i] + len_of(i) + BLK - 1) / BLK);
     }
     SplitPlan plan = plan_split(n_items, current_sm_count(), D,
                                 alike && nkv_max >= kSplitMinBlocks);

@@ -131,6 +131,32 @@ def test_tile_path_host_checks(lib):
              256, None) == ca.CA_ERR_UNSUPPORTED
 
 
+def test_paged_path_host_checks(lib):
+    f = lib.ca_build_kv_pages
+    assert f(A16, 1, 32, 16, 272, 4, A16, A16, None, A16, None) == ca.CA_ERR_INVALID_ARG
+    assert f(A16, 1, 32, 16, 272, 5, A16, A16, A16, A16, None) == ca.CA_ERR_SHAPE
+    assert f(A16, 1, 32, 16, 272, 4, A16, A16, A_MIS, A16, None) == ca.CA_ERR_ALIGN
+    g = lib.ca_paged_chunk_attention
+    cs = (ctypes.c_int32 * 2)(32768, 1024)
+
+    def call(indptr=A16, nnz=100, lens=(2048, 100), L_max=34816):
+        cl = None if lens is None else (ctypes.c_int32 * 2)(*lens)
+        return g(A16, A16, A16, indptr, A16, nnz, cs, cl, 2, 32, 8, 2048, L_max, 128, 128, 0.1,
+                 A16, A16, A16, 256, None)
+    assert call(indptr=None) == ca.CA_ERR_INVALID_ARG
+    assert call(nnz=-1) == ca.CA_ERR_INVALID_ARG
+    assert call(lens=(2049, 100)) == ca.CA_ERR_SHAPE      # longer than C
+    assert call(lens=(-1, 100)) == ca.CA_ERR_SHAPE
+    # a short chunk may sit where a full one would not fit
+    cs2 = (ctypes.c_int32 * 2)(34000, 0)
+    cl2 = (ctypes.c_int32 * 2)(816, 2048)
+    assert g(A16, A16, A16, A16, A16, 10, cs2, cl2, 2, 32, 8, 2048, 34816, 96, 128, 0.1, A16,
+             A16, A16, 256, None) == ca.CA_ERR_UNSUPPORTED   # passes the shape checks, D = 96
+    cl3 = (ctypes.c_int32 * 2)(817, 2048)
+    assert g(A16, A16, A16, A16, A16, 10, cs2, cl3, 2, 32, 8, 2048, 34816, 128, 128, 0.1, A16,
+             A16, A16, 256, None) == ca.CA_ERR_SHAPE
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     monkeypatch.setattr(ca, "_lib", None)
