@@ -102,6 +102,18 @@ constexpr int kSmemFloor = 120 * 1024;  // keeps one CTA (and one TMEM owner) pe
 #define CA_P_CHUNK_KEYS 64
 #endif
 constexpr int kPChunkKeysCfg = CA_P_CHUNK_KEYS;
+
+// Where P (the bf16 probabilities) goes between the softmax and the P.V MMA.
+// 1: shared memory (128B-swizzled, the Q tile layout; P.V reads it as an SS
+// MMA). The S columns in TMEM are free as soon as the softmax has loaded them,
+// so S(j+1) runs on the tensor core while the softmax of block j computes its
+// exponentials. 0: P overwrites S in TMEM (TS-form P.V); S(j+1) then waits
+// for P.V(j) to have read P.
+#ifndef CA_P_SMEM
+#define CA_P_SMEM 0
+#endif
+constexpr bool kPSmem = CA_P_SMEM != 0;
+static_assert(!kPSmem || kColSplit == 1, "P in shared memory needs one softmax warp per row");
 static_assert(kPChunkKeysCfg == 32 || kPChunkKeysCfg == 64 || kPChunkKeysCfg == 128,
               "P chunk must be 32, 64 or 128 keys");
 
@@ -128,20 +140,32 @@ template <int D, int BLK>
 struct Layout {
     static constexpr int kQTile = kTileM * D * 2;  // D/64 sub-tiles of 128 rows x 128 B
     static constexpr int kKV = BLK * D * 2;        // D/64 sub-tiles of BLK rows x 128 B
-    static constexpr int kStagesFit = (kSmemBudget - 2048 - 2 * kQTile) / (2 * kKV);
-    static constexpr int kStages = kStagesFit > 4 ? 4 : kStagesFit;
+    // P tile (shared-memory P only): BLK/64 sub-tiles of 128 rows x 128 B
+    static constexpr int kPTile = kPSmem ? kTileM * BLK * 2 : 0;
+    static constexpr int kXchBytes = kColSplit == 2 ? 2 * 4 * 2 * 32 * 4 : 0;
+    static constexpr int kRoom = kSmemBudget - 2048 - 2 * kQTile - 2 * kPTile - kXchBytes;
+    // K and V ring stages. P in TMEM: equal rings. P in shared memory: K needs
+    // two stages (S(j+1) is issued before P.V(j)), V one fewer when short of room.
+    static constexpr int kFit = kRoom / kKV;  // K + V stages that fit
+    static constexpr int kStagesK = kPSmem ? (kFit >= 8 ? 4 : (kFit + 1) / 2) : (kFit / 2 > 4 ? 4 : kFit / 2);
+    static constexpr int kStagesV = kPSmem ? (kFit - kStagesK > 4 ? 4 : kFit - kStagesK) : kStagesK;
+    static constexpr int kStages = kStagesK;  // ring depth used where K and V agree
     static constexpr int kQOff = 0;
     static constexpr int kKOff = 2 * kQTile;
-    static constexpr int kVOff = kKOff + kStages * kKV;
-    static constexpr int kBarOff = kVOff + kStages * kKV;
+    static constexpr int kVOff = kKOff + kStagesK * kKV;
+    static constexpr int kPOff = kVOff + kStagesV * kKV;
+    static constexpr int kBarOff = kPOff + 2 * kPTile;
     static constexpr int kPChunkKeys =
         kColSplit == 2 ? BLK / 2 : (kPChunkKeysCfg < BLK ? kPChunkKeysCfg : BLK);
     static constexpr int kPChunks = BLK / kPChunkKeys;  // P reaches the MMA chunk by chunk
-    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 * kPChunks + 2 + 1 + 8;
+    static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 2 + 2 * kPChunks + 2 + 1 +
+                                    8 + 2 + 2;
     static constexpr int kXchOff = kBarOff + kNumBars * 8 + 16;  // [2][4][2][32] floats
-    static constexpr int kEnd = kXchOff + 2 * 4 * 2 * 32 * 4;
+    static constexpr int kEnd = kXchOff + kXchBytes;
     static constexpr int kDynamic = (kEnd + 1024) > kSmemFloor ? (kEnd + 1024) : kSmemFloor;
-    static_assert(kStages >= 2, "need at least two K/V stages");
+    static_assert(kStagesK >= 2 && kStagesV >= 1, "need two K stages and a V stage");
+    static_assert(kPSmem || kStagesV >= 2, "need two V stages");
+    static_assert(!kPSmem || kPChunkKeys == 64, "shared-memory P hands over 64-key sub-tiles");
     static_assert(kDynamic <= kSmemBudget, "shared memory budget exceeded");
 };
 
@@ -183,6 +207,18 @@ __device__ __forceinline__ constexpr bool use_poly_pair(int q) {
     return kPolyEvery > 0 && (q % kPolyEvery) == kPolyEvery - 1;
 }
 
+// Stores 64 bf16 probabilities of one row (32 packed pairs: keys 8u .. 8u+7 in
+// pk[4u .. 4u+3]) into row m of a 128-row x 128-byte sub-tile of the P tile,
+// 128B-swizzled like the TMA-loaded Q tile (16-byte unit u of row m sits at
+// unit u ^ (m & 7)), so the P.V MMA reads it with the Q tile's descriptor.
+__device__ __forceinline__ void store_p_chunk(uint8_t *subtile, int m, const uint32_t (&pk)[32]) {
+    uint8_t *row = subtile + m * 128;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+        *reinterpret_cast<uint4 *>(row + ((u ^ (m & 7)) << 4)) =
+            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+}
+
 // Named barrier 1 over the softmax warps only (barrier 0 is __syncthreads).
 __device__ __forceinline__ void softmax_bar_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxWarps * 32) : "memory");
@@ -213,6 +249,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr bool COMPACT = MODE == kModeCompact;  // K/V block t sits at row t * BLK
     constexpr bool PERTILE = MODE == kModePerTile;  // one head per tile, span tables
     constexpr int NST = L::kStages;
+    constexpr int NSK = L::kStagesK;  // K ring
+    constexpr int NSV = L::kStagesV;  // V ring
     constexpr int DCH = D / 64;  // 64-element (128-byte) sub-tiles along D
     constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, BLK, false);
     constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, true);
@@ -225,16 +263,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
     uint64_t *q_full = bars;
     uint64_t *k_full = bars + 1;
-    uint64_t *k_empty = k_full + NST;
-    uint64_t *v_full = k_empty + NST;
-    uint64_t *v_empty = v_full + NST;
+    uint64_t *k_empty = k_full + NSK;
+    uint64_t *v_full = k_empty + NSK;
+    uint64_t *v_empty = v_full + NSV;
     constexpr int NPC = L::kPChunks;
-    uint64_t *s_full = v_empty + NST;   // [2]
+    uint64_t *s_full = v_empty + NSV;   // [2]
     uint64_t *p_full = s_full + 2;      // [2][NPC]: P chunk c of tile t stored in TMEM
     uint64_t *o_full = p_full + 2 * NPC;  // [2]
     uint64_t *mma_done = o_full + 2;
     uint64_t *xch_bar = mma_done + 1;  // [2 tiles][4 quarters]: the two half-row warps meet
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xch_bar + 8);
+    uint64_t *s_free = xch_bar + 8;     // [2] softmax has loaded S (shared-memory P)
+    uint64_t *p_free = s_free + 2;      // [2] P.V of the tile done (shared-memory P)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(p_free + 2);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     int *last_flag = abort_flag + 1;  // split items: this CTA merges the segments
 
@@ -273,9 +313,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < NST; ++s) {
+        for (int s = 0; s < NSK; ++s) {
             mbar_init(k_full + s, 1);
             mbar_init(k_empty + s, 1);
+        }
+        for (int s = 0; s < NSV; ++s) {
             mbar_init(v_full + s, 1);
             mbar_init(v_empty + s, 1);
         }
@@ -286,6 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_init(mma_done, 1);
         for (int x = 0; x < 8; ++x) mbar_init(xch_bar + x, 2);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(s_free + t, 4);
+            mbar_init(p_free + t, 1);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -359,7 +405,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     q_full, dc * 64, r0 + t * R, b * P.H_q + head0);
             }
             q_issued = true;
+            // K(j) into ring stage j % NSK, V(j) into j % NSV (lane 0 only);
+            // false if a wait gave up
+            auto load_k = [&](int j, int blk_idx) -> bool {
+                const int s = j % NSK;
+                if (!mbar_wait(k_empty + s, ((j / NSK) & 1) ^ 1, ab)) return false;
+                mbar_arrive_expect_tx(k_full + s, L::kKV);
+                for (int dc = 0; dc < DCH; ++dc)
+                    tma_load_3d(smem + L::kKOff + s * L::kKV + dc * (BLK * 128), &tmK,
+                                k_full + s, dc * 64, blk_idx * BLK, b * P.H_kv + g);
+                k_issued = j + 1;
+                return true;
+            };
+            auto load_v = [&](int j, int blk_idx) -> bool {
+                const int s = j % NSV;
+                if (!mbar_wait(v_empty + s, ((j / NSV) & 1) ^ 1, ab)) return false;
+                mbar_arrive_expect_tx(v_full + s, L::kKV);
+                for (int dc = 0; dc < DCH; ++dc)
+                    tma_load_3d(smem + L::kVOff + s * L::kKV + dc * (BLK * 128), &tmV,
+                                v_full + s, dc * 64, blk_idx * BLK, b * P.H_kv + g);
+                v_issued = j + 1;
+                return true;
+            };
             int prev_last = -1;
+            int prev_blk = 0;  // block of the previous K load (lane 0)
             bool ok = true;
             for (int w0 = 0; w0 < n_run && ok; w0 += 32) {
                 const int jj = t0 + w0 + lane;  // table index
@@ -379,26 +448,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int q = 0; q < nwin; ++q) {
                     const int j = w0 + q;
                     const int blk_idx = COMPACT ? t0 + j : __shfl_sync(0xffffffffu, jb, q);
-                    const int s = j % NST;
-                    const uint32_t ph = ((j / NST) & 1) ^ 1;
                     int good = 1;
                     if (lane == 0) {
-                        good = mbar_wait(k_empty + s, ph, ab);
+                        // with P in shared memory, K runs one block ahead of V:
+                        // S(j + 1) is issued before P.V(j)
+                        good = load_k(j, blk_idx);
                         if (good) {
-                            mbar_arrive_expect_tx(k_full + s, L::kKV);
-                            for (int dc = 0; dc < DCH; ++dc)
-                                tma_load_3d(smem + L::kKOff + s * L::kKV + dc * (BLK * 128), &tmK,
-                                            k_full + s, dc * 64, blk_idx * BLK, b * P.H_kv + g);
-                            k_issued = j + 1;
-                            good = mbar_wait(v_empty + s, ph, ab);
+                            if (kPSmem) {
+                                if (j > 0) good = load_v(j - 1, prev_blk);
+                            } else {
+                                good = load_v(j, blk_idx);
+                            }
                         }
-                        if (good) {
-                            mbar_arrive_expect_tx(v_full + s, L::kKV);
-                            for (int dc = 0; dc < DCH; ++dc)
-                                tma_load_3d(smem + L::kVOff + s * L::kKV + dc * (BLK * 128), &tmV,
-                                            v_full + s, dc * 64, blk_idx * BLK, b * P.H_kv + g);
-                            v_issued = j + 1;
-                        }
+                        prev_blk = blk_idx;
                     }
                     good = __shfl_sync(0xffffffffu, good, 0);
                     if (!good) {
@@ -407,14 +469,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
+            if (kPSmem && ok && lane == 0) load_v(n_run - 1, prev_blk);
         }
         // drain: every copy this warp started has landed before the CTA exits
         if (lane == 0) {
             if (q_issued) mbar_wait_drain(q_full, 0);
-            for (int j = k_issued > NST ? k_issued - NST : 0; j < k_issued; ++j)
-                mbar_wait_drain(k_full + j % NST, (j / NST) & 1);
-            for (int j = v_issued > NST ? v_issued - NST : 0; j < v_issued; ++j)
-                mbar_wait_drain(v_full + j % NST, (j / NST) & 1);
+            for (int j = k_issued > NSK ? k_issued - NSK : 0; j < k_issued; ++j)
+                mbar_wait_drain(k_full + j % NSK, (j / NSK) & 1);
+            for (int j = v_issued > NSV ? v_issued - NSV : 0; j < v_issued; ++j)
+                mbar_wait_drain(v_full + j % NSV, (j / NSV) & 1);
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -461,6 +524,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 return true;
             };
+            // P.V of tile t with P read from shared memory (64-key sub-tile c of
+            // the P tile is chunk c); false if a wait gave up.
+            const uint64_t dp = sdesc_sw128(sbase + L::kPOff, 16, 1024);
+            const uint32_t p_lo = static_cast<uint32_t>(dp), p_hi = static_cast<uint32_t>(dp >> 32);
+            auto issue_pv_smem = [&](int t, int slot, bool acc, uint32_t par) -> bool {
+                const uint32_t a0 = p_lo + t * (L::kPTile >> 4);
+                const uint32_t b0 = v_lo + slot * kStageUnits;
+#pragma unroll
+                for (int c = 0; c < NPC; ++c) {
+                    if (!mbar_wait(p_full + t * NPC + c, par, ab)) return false;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 4 * c; kk < 4 * c + 4; ++kk) {
+                        const uint32_t ao = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
+                        mma_ss_w(tmem + 256 + t * 128, a0 + ao, p_hi,
+                                 b0 + ((kk * (16 * 128)) >> 4), v_hi, kIdescPV,
+                                 (acc || kk > 0) ? 1u : 0u);
+                    }
+                }
+                return true;
+            };
             bool ok = mbar_wait(q_full, 0, ab) && mbar_wait(k_full, 0, ab);
             if (ok) {
                 tc_fence_after();
@@ -470,7 +554,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_commit(s_full + 1);
                 tc_commit(k_empty + 0);
             }
-            for (int j = 0; j < n_run && ok; ++j) {
+            // P in shared memory: per block j, S(j + 1) of both tiles (as soon as
+            // each tile's softmax has loaded S(j)), then P.V(j) of both tiles.
+            for (int j = 0; kPSmem && j < n_run && ok; ++j) {
+                const bool more = j + 1 < n_run;
+                if (more) {
+                    const int ks = (j + 1) % NSK;
+                    if (!(ok = mbar_wait(k_full + ks, ((j + 1) / NSK) & 1, ab))) break;
+                    if (!(ok = mbar_wait(s_free + 0, j & 1, ab))) break;
+                    tc_fence_after();
+                    issue_s(0, ks);
+                    tc_commit(s_full + 0);
+                    if (!(ok = mbar_wait(s_free + 1, j & 1, ab))) break;
+                    tc_fence_after();
+                    issue_s(1, ks);
+                    tc_commit(s_full + 1);
+                    tc_commit(k_empty + ks);
+                }
+                const int vs = j % NSV;
+                if (!(ok = mbar_wait(v_full + vs, (j / NSV) & 1, ab))) break;
+                if (!(ok = issue_pv_smem(0, vs, j > 0, j & 1))) break;
+                tc_commit(p_free + 0);
+                if (!more) tc_commit(o_full + 0);
+                if (!(ok = issue_pv_smem(1, vs, j > 0, j & 1))) break;
+                tc_commit(p_free + 1);
+                if (!more) tc_commit(o_full + 1);
+                tc_commit(v_empty + vs);
+            }
+            for (int j = 0; !kPSmem && j < n_run && ok; ++j) {
                 const int s = j % NST;
                 const uint32_t ph = (j / NST) & 1;
                 const bool more = j + 1 < n_run;
@@ -561,16 +672,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t zero[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) zero[i] = 0u;
-#pragma unroll
-                for (int cl = 0; cl < CPW; ++cl) {
-                    constexpr int CK = L::kPChunkKeys;
-                    const int c = hf * CPW + cl;
-#pragma unroll
-                    for (int q = 0; q < CK / 32; ++q) tmem_st16(tS + c * (CK / 2) + q * 16, zero);
-                    tmem_st_wait();
+                if constexpr (kPSmem) {
+                    // S(j) is not needed: release its columns, then zero this
+                    // row of the P tile once P.V(j - 1) has read it
                     tc_fence_before();
                     __syncwarp();
-                    mbar_arrive_lane0(p_full + t * NPC + c, lane);
+                    mbar_arrive_lane0(s_free + t, lane);
+                    if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(p_free + t, (j - 1) & 1, ab))) {
+                        ok = false;
+                        break;
+                    }
+                    uint32_t z32[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) z32[i] = 0u;
+#pragma unroll
+                    for (int c = 0; c < NPC; ++c) {
+                        store_p_chunk(smem + L::kPOff + t * L::kPTile + c * (kTileM * 128), m, z32);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        mbar_arrive_lane0(p_full + t * NPC + c, lane);
+                    }
+                } else {
+#pragma unroll
+                    for (int cl = 0; cl < CPW; ++cl) {
+                        constexpr int CK = L::kPChunkKeys;
+                        const int c = hf * CPW + cl;
+#pragma unroll
+                        for (int q = 0; q < CK / 32; ++q)
+                            tmem_st16(tS + c * (CK / 2) + q * 16, zero);
+                        tmem_st_wait();
+                        tc_fence_before();
+                        __syncwarp();
+                        mbar_arrive_lane0(p_full + t * NPC + c, lane);
+                    }
                 }
                 continue;
             }
@@ -580,6 +714,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_row<CW>(tS + hf * CW, v);  // this warp's S columns in one round trip
 #pragma unroll
                 for (int i = 0; i < CW; ++i) s[i] = __uint_as_float(v[i]);
+            }
+            if constexpr (kPSmem) {
+                // S(j) is in registers: its TMEM columns can take S(j + 1)
+                tc_fence_before();
+                __syncwarp();
+                mbar_arrive_lane0(s_free + t, lane);
             }
             if (t0 + j >= n_full) {
                 int jb = DENSE ? t0 + j : (PERTILE ? block_of<true>(e_j) : __ldg(T + t0 + j) - base);
@@ -626,7 +766,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // before the first P chunk is handed over. Each warp rescales its
             // DW columns of O.
             const bool need = upd && old_finite && j > 0;
-            if (__any_sync(0xffffffffu, need)) {
+            // (with P in shared memory the rescale waits for P.V(j - 1) first; it
+            // runs inside the chunk loop below)
+            if (!kPSmem && __any_sync(0xffffffffu, need)) {
                 const float a = need ? alpha : 1.0f;
 #pragma unroll
                 for (int c = 0; c < DW / 16; ++c) {
@@ -662,13 +804,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                     acc2[i & 3] = f2_add(acc2[i & 3], p2);
                     pk[i] = pack_bf16x2(f2_lo(p2), f2_hi(p2));
                 }
+                if constexpr (kPSmem) {
+                    if (cl == 0 && j > 0) {
+                        // P.V(j - 1) must have read this tile's P (and finished
+                        // with O) before P(j) and any O rescale land
+                        if (!__all_sync(0xffffffffu, mbar_wait(p_free + t, (j - 1) & 1, ab))) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        if (__any_sync(0xffffffffu, need)) {
+                            const float a = need ? alpha : 1.0f;
 #pragma unroll
-                for (int q = 0; q < CK / 32; ++q) tmem_st16(tS + c * (CK / 2) + q * 16, pk + q * 16);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                mbar_arrive_lane0(p_full + t * NPC + c, lane);
+                            for (int oc = 0; oc < DW / 16; ++oc) {
+                                uint32_t v[16];
+                                tmem_ld16(tO + oc * 16, v);
+#pragma unroll
+                                for (int i = 0; i < 16; ++i)
+                                    v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
+                                tmem_st16(tO + oc * 16, v);
+                            }
+                            tmem_st_wait();
+                            tc_fence_before();
+                        }
+                    }
+                    store_p_chunk(smem + L::kPOff + t * L::kPTile + c * (kTileM * 128), m, pk);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    mbar_arrive_lane0(p_full + t * NPC + c, lane);
+                } else {
+#pragma unroll
+                    for (int q = 0; q < CK / 32; ++q)
+                        tmem_st16(tS + c * (CK / 2) + q * 16, pk + q * 16);
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    mbar_arrive_lane0(p_full + t * NPC + c, lane);
+                }
             }
+            if (!ok) break;
             acc2[0] = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
             const float sum = f2_lo(acc2[0]) + f2_hi(acc2[0]);
             l_run += sum;
