@@ -76,6 +76,18 @@ int ca_build_block_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVma
                           int32_t *tables, int32_t *counts, int32_t *indptr, int32_t *indices,
                           void *stream);
 
+/*
+ * ca_build_block_tables from a bit-packed mask: mask_bits uint32
+ * [B, H_q, nQ, ceil(nKVmax / 32)], bit k (value 1 << k) of word w selects KV
+ * block 32 * w + k; bits naming blocks at or past nKVmax are ignored. Eight
+ * times less mask traffic than the byte mask. Outputs, errors and results are
+ * those of ca_build_block_tables for the equivalent byte mask (mask_bits must
+ * be 4-byte aligned).
+ */
+int ca_build_block_tables_bits(const uint32_t *mask_bits, int B, int H_q, int nQ, int nKVmax,
+                               int group, int32_t *tables, int32_t *counts, int32_t *indptr,
+                               int32_t *indices, void *stream);
+
 /* Bytes of device workspace the attention entry points use for these sizes on
  * the current device, for D <= 128: a 256-byte header (status word) plus room
  * for the split of the last wave of work items (split-KV: when the items do

@@ -71,6 +71,7 @@ EXPORTED_SYMBOLS = (
     "ca_compacted_chunk_attention",
     "ca_tile_span",
     "ca_build_kv_pages",
+    "ca_build_block_tables_bits",
     "ca_paged_chunk_attention",
     "ca_build_tile_tables",
     "ca_tile_chunk_attention",
@@ -122,6 +123,8 @@ def load_library():
         lib.ca_compacted_chunk_attention.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P,
                                                      P, P, S, P]
         lib.ca_compacted_chunk_attention.restype = I
+        lib.ca_build_block_tables_bits.argtypes = [P, I, I, I, I, I, P, P, P, P, P]
+        lib.ca_build_block_tables_bits.restype = I
         lib.ca_build_kv_pages.argtypes = [P, I, I, I, I, I, P, P, P, P, P]
         lib.ca_build_kv_pages.restype = I
         lib.ca_paged_chunk_attention.argtypes = [P, P, P, P, P, ctypes.c_longlong, P, P, I, I, I,
@@ -215,6 +218,44 @@ def build_block_tables(mask: torch.Tensor, group: int, csr: bool = False,
                                    _ptr(counts), _ptr(indptr), _ptr(indices),
                                    _stream_handle(stream, dev))
     _check("ca_build_block_tables", st)
+    return tables, counts, indptr, indices
+
+
+def build_block_tables_bits(mask_bits: torch.Tensor, nKVmax: int, group: int, csr: bool = False,
+                            tables: Optional[torch.Tensor] = None,
+                            counts: Optional[torch.Tensor] = None,
+                            stream: Optional[torch.cuda.Stream] = None):
+    """Block-Union tables from a bit-packed mask ``int32/uint32 [B, H_q, nQ,
+    ceil(nKVmax/32)]`` (bit k of word w selects block 32*w + k); the same
+    outputs as :func:`build_block_tables`."""
+    if mask_bits.dtype not in (torch.int32, torch.uint32):
+        raise TypeError("mask_bits must be int32 or uint32")
+    if mask_bits.dim() != 4 or not mask_bits.is_cuda or not mask_bits.is_contiguous():
+        raise ValueError("mask_bits must be a contiguous 4-D CUDA tensor")
+    B, H_q, nQ, nW = mask_bits.shape
+    if nW != -(-nKVmax // 32):
+        raise ValueError("last dim must be ceil(nKVmax / 32)")
+    if group <= 0 or H_q % group:
+        raise ValueError("group must divide H_q")
+    H_kv = H_q // group
+    dev = mask_bits.device
+    if tables is None:
+        tables = torch.empty((B, H_kv, nKVmax), dtype=torch.int32, device=dev)
+    if counts is None:
+        counts = torch.empty((B, H_kv), dtype=torch.int32, device=dev)
+    _need(tables, "tables", torch.int32, 3)
+    _need(counts, "counts", torch.int32, 2)
+    if tuple(tables.shape) != (B, H_kv, nKVmax) or tuple(counts.shape) != (B, H_kv):
+        raise ValueError(f"tables must be {(B, H_kv, nKVmax)}, counts {(B, H_kv)}")
+    indptr = indices = None
+    if csr:
+        indptr = torch.empty(B * H_kv + 1, dtype=torch.int32, device=dev)
+        indices = torch.empty(B * H_kv * nKVmax, dtype=torch.int32, device=dev)
+    st = load_library().ca_build_block_tables_bits(_ptr(mask_bits), B, H_q, nQ, int(nKVmax),
+                                                   int(group), _ptr(tables), _ptr(counts),
+                                                   _ptr(indptr), _ptr(indices),
+                                                   _stream_handle(stream, dev))
+    _check("ca_build_block_tables_bits", st)
     return tables, counts, indptr, indices
 
 

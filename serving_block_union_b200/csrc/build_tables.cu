@@ -137,6 +137,67 @@ __global__ void __launch_bounds__(kMaxThreads)
     if (tid == 0) counts[bg] = n;
 }
 
+// The same union from a bit-packed mask: uint32 words [B, H_q, nQ, nW],
+// nW = ceil(nKVmax / 32), bit k of word w selects KV block 32 * w + k (bits
+// at or past nKVmax are ignored). Thread (r_grp, w) ORs word w of rows
+// r_grp, r_grp + rg, ...; the row groups combine through shared memory and a
+// block-wide scan of the popcounts places each word's blocks.
+__global__ void __launch_bounds__(kMaxThreads)
+    union_bits_kernel(const uint32_t *__restrict__ mask, int H_q, int nQ, int nKVmax, int G,
+                      int wpr, int rg, int32_t *__restrict__ tables,
+                      int32_t *__restrict__ counts) {
+    extern __shared__ uint32_t sm_words[];  // [rg][wpr]
+    __shared__ int warp_sums[32];
+    __shared__ int s_base;
+
+    const int bg = blockIdx.x;
+    const int H_kv = H_q / G;
+    const int b = bg / H_kv, g = bg % H_kv;
+    const int tid = threadIdx.x;
+    const int w_local = tid % wpr, r_grp = tid / wpr;
+    const int n_rows = G * nQ;
+    const int nW = (nKVmax + 31) >> 5;
+    const uint32_t *base = mask + ((size_t)b * H_q + (size_t)g * G) * nQ * (size_t)nW;
+    int32_t *T = tables + (size_t)bg * nKVmax;
+
+    if (tid == 0) s_base = 0;
+    __syncthreads();
+
+    for (int round0 = 0; round0 < nW; round0 += wpr) {
+        const int w = round0 + w_local;
+        uint32_t bits = 0;
+        if (w < nW) {
+#pragma unroll 8
+            for (int row = r_grp; row < n_rows; row += rg) bits |= __ldg(base + (size_t)row * nW + w);
+            const int valid = nKVmax - (w << 5);  // blocks this word can name
+            if (valid < 32) bits &= (1u << valid) - 1u;
+        }
+        sm_words[r_grp * wpr + w_local] = bits;
+        __syncthreads();
+        int total = 0;
+        if (r_grp == 0) {
+            for (int q = 1; q < rg; ++q) bits |= sm_words[q * wpr + w_local];
+        }
+        const int cnt = (r_grp == 0) ? __popc(bits) : 0;
+        const int off = block_exclusive_scan(cnt, tid, wpr * rg, warp_sums, &total);
+        if (r_grp == 0 && bits) {
+            int o = s_base + off;
+            uint32_t m = bits;
+            while (m) {
+                const int k = __ffs(m) - 1;
+                T[o++] = (w << 5) + k;
+                m &= m - 1;
+            }
+        }
+        __syncthreads();
+        if (tid == 0) s_base += total;
+        __syncthreads();
+    }
+    const int n = s_base;
+    for (int t = n + tid; t < nKVmax; t += blockDim.x) T[t] = -1;
+    if (tid == 0) counts[bg] = n;
+}
+
 // CSR form: indptr[bg] = sum of counts before bg; indices = valid prefixes.
 __global__ void __launch_bounds__(256)
     csr_kernel(const int32_t *__restrict__ tables, const int32_t *__restrict__ counts, int n_bg,
@@ -166,7 +227,32 @@ __global__ void __launch_bounds__(256)
     }
 }
 
+int launch_csr(const int32_t *tables, const int32_t *counts, int n_bg, int nKVmax,
+               bool page_ids, int32_t *indptr, int32_t *indices, cudaStream_t stream) {
+    if (!indptr) return CA_OK;
+    csr_kernel<<<n_bg, 256, 0, stream>>>(tables, counts, n_bg, nKVmax, page_ids, indptr, indices);
+    return cudaGetLastError() == cudaSuccess ? CA_OK : CA_ERR_CUDA;
+}
+
 }  // namespace
+
+int launch_build_tables_bits(const uint32_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
+                             int32_t *tables, int32_t *counts, int32_t *indptr, int32_t *indices,
+                             bool page_ids, cudaStream_t stream) {
+    const int H_kv = H_q / group;
+    const int nW = (nKVmax + 31) / 32;
+    int wpr = ((nW + 31) / 32) * 32;
+    if (wpr > kMaxThreads) wpr = kMaxThreads;
+    int rg = 512 / wpr;
+    if (rg < 1) rg = 1;
+    if (rg > group * nQ) rg = group * nQ;
+    const int threads = wpr * rg;
+    const size_t smem = sizeof(uint32_t) * (size_t)threads;
+    union_bits_kernel<<<B * H_kv, threads, smem, stream>>>(mask, H_q, nQ, nKVmax, group, wpr, rg,
+                                                            tables, counts);
+    if (cudaGetLastError() != cudaSuccess) return CA_ERR_CUDA;
+    return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
+}
 
 int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
                         int32_t *tables, int32_t *counts, int32_t *indptr, int32_t *indices,
@@ -186,15 +272,8 @@ int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax,
     const size_t smem = sizeof(uint32_t) * (size_t)threads;
     union_tables_kernel<<<B * H_kv, threads, smem, stream>>>(mask, H_q, nQ, nKVmax, group, chp,
                                                               rg, vec, tables, counts);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return CA_ERR_CUDA;
-    if (indptr) {
-        csr_kernel<<<B * H_kv, 256, 0, stream>>>(tables, counts, B * H_kv, nKVmax, page_ids,
-                                                  indptr, indices);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return CA_ERR_CUDA;
-    }
-    return CA_OK;
+    if (cudaGetLastError() != cudaSuccess) return CA_ERR_CUDA;
+    return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
 }
 
 }  // namespace ca

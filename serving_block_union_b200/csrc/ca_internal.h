@@ -21,6 +21,11 @@ int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax,
                         int32_t *tables, int32_t *counts, int32_t *indptr, int32_t *indices,
                         bool page_ids, cudaStream_t stream);
 
+// The same from a bit-packed mask (uint32 [B, H_q, nQ, ceil(nKVmax / 32)]).
+int launch_build_tables_bits(const uint32_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
+                             int32_t *tables, int32_t *counts, int32_t *indptr, int32_t *indices,
+                             bool page_ids, cudaStream_t stream);
+
 struct AttnArgs {
     const void *Q, *K, *V;
     const int32_t *tables, *counts;  // NULL for the dense path

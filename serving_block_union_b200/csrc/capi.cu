@@ -100,6 +100,23 @@ int ca_build_block_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVma
                                    indices, false, static_cast<cudaStream_t>(stream));
 }
 
+int ca_build_block_tables_bits(const uint32_t *mask_bits, int B, int H_q, int nQ, int nKVmax,
+                               int group, int32_t *tables, int32_t *counts, int32_t *indptr,
+                               int32_t *indices, void *stream) {
+    if (!mask_bits || !tables || !counts) return CA_ERR_INVALID_ARG;
+    if (indices && !indptr) return CA_ERR_INVALID_ARG;
+    if (B <= 0 || H_q <= 0 || nQ <= 0 || nKVmax <= 0 || group <= 0) return CA_ERR_INVALID_ARG;
+    if (H_q % group != 0) return CA_ERR_SHAPE;
+    if ((long long)B * H_q * nQ * ((nKVmax + 31) / 32) >= (1LL << 38)) return CA_ERR_SHAPE;
+    if ((long long)B * (H_q / group) * nKVmax >= (1LL << 31)) return CA_ERR_SHAPE;
+    if (!aligned(mask_bits, 4) || !aligned(tables, 4) || !aligned(counts, 4) ||
+        (indptr && !aligned(indptr, 4)) || (indices && !aligned(indices, 4)))
+        return CA_ERR_ALIGN;
+    return ca::launch_build_tables_bits(mask_bits, B, H_q, nQ, nKVmax, group, tables, counts,
+                                        indptr, indices, false,
+                                        static_cast<cudaStream_t>(stream));
+}
+
 int ca_build_kv_pages(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
                       int32_t *tables, int32_t *counts, int32_t *kv_indptr, int32_t *kv_indices,
                       void *stream) {

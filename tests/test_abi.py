@@ -131,6 +131,15 @@ def test_tile_path_host_checks(lib):
              256, None) == ca.CA_ERR_UNSUPPORTED
 
 
+def test_bits_build_host_checks(lib):
+    f = lib.ca_build_block_tables_bits
+    assert f(None, 1, 32, 16, 272, 4, A16, A16, None, None, None) == ca.CA_ERR_INVALID_ARG
+    assert f(A16, 1, 32, 16, 272, 3, A16, A16, None, None, None) == ca.CA_ERR_SHAPE
+    assert f(ctypes.c_void_p((1 << 20) + 2), 1, 32, 16, 272, 4, A16, A16, None, None,
+             None) == ca.CA_ERR_ALIGN
+    assert f(A16, 1, 32, 16, 272, 4, A16, A16, None, A16, None) == ca.CA_ERR_INVALID_ARG
+
+
 def test_paged_path_host_checks(lib):
     f = lib.ca_build_kv_pages
     assert f(A16, 1, 32, 16, 272, 4, A16, A16, None, A16, None) == ca.CA_ERR_INVALID_ARG

@@ -46,6 +46,21 @@ def test_bench_tile_visible_pairs_matches_token_count():
     assert bench.tile_visible_pairs(mask, cs, C, blk) == total
 
 
+def test_pack_mask_bits_round_trip():
+    """The bit-packed mask input: bit k of word w is block 32*w + k, any
+    nonzero byte selects, bits past nKVmax stay clear (checked bit by bit
+    with Python integers, independent of numpy's packing)."""
+    rng = np.random.default_rng(9)
+    for nK in (1, 31, 32, 33, 95):
+        m = (rng.random((2, 2, 3, nK)) < 0.4).astype(np.uint8) * 3
+        w = workloads.pack_mask_bits(m)
+        assert w.dtype == np.uint32 and w.shape == (2, 2, 3, -(-nK // 32))
+        for idx in np.ndindex(m.shape[:3]):
+            value = sum(1 << j for j in range(nK) if m[idx + (j,)])
+            words = [int(x) for x in w[idx]]
+            assert sum(x << (32 * i) for i, x in enumerate(words)) == value
+
+
 def _poly_coeffs():
     src = open(os.path.join(ROOT, "serving_block_union_b200", "csrc", "sm100_ptx.cuh")).read()
     body = src[src.index("float exp2_poly(float x)"):]

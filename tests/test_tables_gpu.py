@@ -81,3 +81,37 @@ def test_tables_stream_ordering(cuda_ok):
     T_ref, c_ref, _, _ = oracle.block_tables(mask, wl.group)
     np.testing.assert_array_equal(T.cpu().numpy(), T_ref)
     np.testing.assert_array_equal(c.cpu().numpy(), c_ref)
+
+
+
+@pytest.mark.parametrize("name", WORKLOADS)
+def test_bit_packed_mask_gives_the_same_tables(cuda_ok, name):
+    """The bit-packed input (uint32 words) yields the byte mask's tables and
+    CSR, bit for bit."""
+    wl = workloads.by_name(name)
+    mask = workloads.make_mask(wl)
+    words = torch.from_numpy(workloads.pack_mask_bits(mask).view(np.int32)).cuda()
+    T, c, ip, ix = ca.build_block_tables_bits(words, wl.nKVmax, wl.group, csr=True)
+    T_ref, c_ref, ip_ref, ix_ref = oracle.block_tables(mask, wl.group)
+    np.testing.assert_array_equal(T.cpu().numpy(), T_ref)
+    np.testing.assert_array_equal(c.cpu().numpy(), c_ref)
+    np.testing.assert_array_equal(ip.cpu().numpy(), ip_ref)
+    n = int(ip_ref[-1])
+    np.testing.assert_array_equal(ix.cpu().numpy()[:n], ix_ref[:n])
+
+
+@pytest.mark.parametrize("shape", [(1, 4, 3, 33, 1), (2, 8, 5, 64, 4), (1, 16, 2, 1, 8),
+                                   (3, 6, 7, 100, 2)])
+def test_bit_packed_random_masks(cuda_ok, shape):
+    B, H_q, nQ, nK, G = shape
+    rng = np.random.default_rng(sum(shape))
+    mask = (rng.random((B, H_q, nQ, nK)) < 0.1).astype(np.uint8)
+    words = workloads.pack_mask_bits(mask)
+    # garbage in the bits past nKVmax must be ignored
+    tail = (-nK) % 32
+    if tail:
+        words[..., -1] |= np.uint32(((1 << tail) - 1) << (32 - tail))
+    T, c, _, _ = ca.build_block_tables_bits(torch.from_numpy(words.view(np.int32)).cuda(), nK, G)
+    T_ref, c_ref, _, _ = oracle.block_tables(mask, G)
+    np.testing.assert_array_equal(T.cpu().numpy(), T_ref)
+    np.testing.assert_array_equal(c.cpu().numpy(), c_ref)

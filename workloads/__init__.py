@@ -46,6 +46,7 @@ __all__ = [
     "make_q",
     "make_kv",
     "poison_beyond_kv_len",
+    "pack_mask_bits",
 ]
 
 
@@ -310,3 +311,16 @@ def poison_beyond_kv_len(wl: Workload, K: torch.Tensor, V: torch.Tensor) -> None
 
 def chunk_starts(wl: Workload) -> List[int]:
     return list(wl.chunk_start)
+
+
+def pack_mask_bits(mask: np.ndarray) -> np.ndarray:
+    """Bit-packed form of a block mask (an input encoding, no method
+    arithmetic): uint32 ``[B, H_q, nQ, ceil(nKVmax / 32)]``, bit k (value
+    ``1 << k``) of word w set iff ``mask[..., 32 * w + k] != 0``; bits past
+    nKVmax are zero."""
+    B, H, nQ, nK = mask.shape
+    nW = -(-nK // 32)
+    padded = np.zeros((B, H, nQ, nW * 32), dtype=bool)
+    padded[..., :nK] = mask != 0
+    bytes_ = np.packbits(padded.reshape(B, H, nQ, nW, 4, 8), axis=-1, bitorder="little")
+    return bytes_.reshape(B, H, nQ, nW, 4).copy().view("<u4").reshape(B, H, nQ, nW)
