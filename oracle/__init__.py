@@ -53,6 +53,12 @@ def _load():
                                                        ctypes.c_double, P, ctypes.c_int64, P, P,
                                                        I]
             lib.oracle_attention_tile_rows.restype = I
+            lib.oracle_attention_rows_e4m3.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I,
+                                                       ctypes.c_double, P, ctypes.c_int64, P, P,
+                                                       I]
+            lib.oracle_attention_rows_e4m3.restype = I
+            lib.oracle_e4m3_decode.argtypes = [I]
+            lib.oracle_e4m3_decode.restype = ctypes.c_double
             lib.oracle_tile_span_tables.argtypes = [P, I, I, I, I, I, P, P]
             lib.oracle_tile_span_tables.restype = I
             lib.oracle_visible_pairs.argtypes = [P, P, P, I, I, I, I, I, I]
@@ -134,6 +140,62 @@ def attention(Q, K, V, chunk_start: Sequence[int], blk: int, tables=None, counts
                                        n, _ptr(O), _ptr(LSE), int(threads))
     if st != 0:
         raise ValueError(f"oracle_attention_rows failed ({st})")
+    if rows is None:
+        return O.reshape(B, H_q, C, D), LSE.reshape(B, H_q, C)
+    return O, LSE
+
+
+def _u8(t) -> np.ndarray:
+    """uint8 codes of a torch uint8 / float8_e4m3fn tensor or a numpy array."""
+    if hasattr(t, "detach"):
+        import torch
+        t = t.detach().cpu().contiguous()
+        if t.dtype != torch.uint8:
+            t = t.view(torch.uint8)
+        return t.numpy()
+    return np.ascontiguousarray(t, dtype=np.uint8)
+
+
+def e4m3_decode(code: int) -> float:
+    """The real value of one FP8 E4M3 code (0..255)."""
+    return float(_load().oracle_e4m3_decode(int(code)))
+
+
+def attention_e4m3(Q8, K8, V8, descale: Sequence[float], chunk_start: Sequence[int], blk: int,
+                   tables=None, counts=None, scale: Optional[float] = None,
+                   rows: Optional[np.ndarray] = None,
+                   threads: int = 0) -> Tuple[np.ndarray, np.ndarray]:
+    """fp64 chunk attention on FP8 inputs: the real Q, K, V are
+    ``descale[0] * Q8``, ``descale[1] * K8``, ``descale[2] * V8`` with the
+    E4M3 codes decoded exactly. Shapes and results as :func:`attention`."""
+    q, k, v = _u8(Q8), _u8(K8), _u8(V8)
+    B, H_q, C, D = q.shape
+    Bk, H_kv, L_max, Dk = k.shape
+    if Bk != B or Dk != D or v.shape != k.shape:
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = 1.0 / float(np.sqrt(D))
+    ds = np.ascontiguousarray(descale, dtype=np.float64)
+    if ds.shape != (3,):
+        raise ValueError("descale must hold the Q, K and V factors")
+    cs = np.ascontiguousarray(chunk_start, dtype=np.int32)
+    t = c = None
+    if tables is not None:
+        t = np.ascontiguousarray(tables, dtype=np.int32)
+        c = np.ascontiguousarray(counts, dtype=np.int32)
+    r = None
+    n = B * H_q * C
+    if rows is not None:
+        r = np.ascontiguousarray(rows, dtype=np.int64)
+        n = r.size
+    O = np.empty((n, D), np.float64)
+    LSE = np.empty(n, np.float64)
+    st = _load().oracle_attention_rows_e4m3(_ptr(q), _ptr(k), _ptr(v), _ptr(ds), _ptr(t), _ptr(c),
+                                            _ptr(cs), B, H_q, H_kv, C, L_max, D, blk,
+                                            float(scale), _ptr(r), n, _ptr(O), _ptr(LSE),
+                                            int(threads))
+    if st != 0:
+        raise ValueError(f"oracle_attention_rows_e4m3 failed ({st})")
     if rows is None:
         return O.reshape(B, H_q, C, D), LSE.reshape(B, H_q, C)
     return O, LSE

@@ -42,6 +42,23 @@
 #define ORACLE_ENOMEM (-3)
 
 /* bf16 is the top half of an IEEE binary32: widening is exact. */
+/* FP8 E4M3 (the OCP 8-bit format without infinities): sign bit, 4 exponent
+ * bits with bias 7, 3 mantissa bits. Exponent field 0 holds the subnormals
+ * m/8 * 2^-6; the code with every exponent and mantissa bit set is NaN;
+ * everything else is (1 + m/8) * 2^(e - 7). The largest finite value is 448. */
+static double e4m3_to_f64(uint8_t bits) {
+    const int sign = bits >> 7, e = (bits >> 3) & 15, m = bits & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m / 8.0, -6);
+    else
+        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+double oracle_e4m3_decode(int bits) { return e4m3_to_f64((uint8_t)(bits & 0xFF)); }
+
 static double bf16_to_f64(uint16_t bits) {
     uint32_t u = ((uint32_t)bits) << 16;
     float f;
@@ -100,7 +117,9 @@ int oracle_block_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax,
 /* ---------------------------------------------------------------------- */
 
 typedef struct {
-    const uint16_t *Q, *K, *V;       /* bf16 bits */
+    const void *Q, *K, *V;           /* bf16 bits, or e4m3 bytes (fp8) */
+    int fp8;                         /* inputs are e4m3, value = descale * code */
+    double q_descale, k_descale, v_descale;
     const int32_t *tables, *counts;  /* NULL tables: dense, T = [0, nKV_b) */
     const uint8_t *tile_mask;        /* non-NULL: per-tile block-sparse key sets */
     int nQ;                          /* Q-blocks per chunk (tile_mask only) */
@@ -117,6 +136,13 @@ typedef struct {
 static int attention_over_keys(const attn_job *J, int b, int h, int g, int r,
                                const int32_t *keys, int64_t nk, double *s, double *o,
                                double *lse);
+
+/* Element i of an input tensor as a real number: a bf16 value, or an e4m3
+ * code times the tensor's descale factor. */
+static double elem(const void *base, size_t i, int fp8, double descale) {
+    if (fp8) return descale * e4m3_to_f64(((const uint8_t *)base)[i]);
+    return bf16_to_f64(((const uint16_t *)base)[i]);
+}
 
 /* One query row: the definition written out.
  *   K_set = { k : floor(k / blk) in T_{b,g}, k <= p }
@@ -179,9 +205,8 @@ static int attention_over_keys(const attn_job *J, int b, int h, int g, int r,
                                const int32_t *keys, int64_t nk, double *s, double *o,
                                double *lse) {
     const int C = J->C, D = J->D;
-    const uint16_t *q = J->Q + (((size_t)b * J->H_q + h) * C + r) * D;
-    const uint16_t *Kbg = J->K + ((size_t)b * J->H_kv + g) * (size_t)J->L_max * D;
-    const uint16_t *Vbg = J->V + ((size_t)b * J->H_kv + g) * (size_t)J->L_max * D;
+    const size_t q0 = (((size_t)b * J->H_q + h) * C + r) * D;
+    const size_t kv0 = ((size_t)b * J->H_kv + g) * (size_t)J->L_max * D;
 
     if (nk == 0) {
         for (int d = 0; d < D; ++d) o[d] = 0.0;
@@ -190,9 +215,10 @@ static int attention_over_keys(const attn_job *J, int b, int h, int g, int r,
     }
     double m = -INFINITY;
     for (int64_t i = 0; i < nk; ++i) {
-        const uint16_t *kr = Kbg + (size_t)keys[i] * D;
+        const size_t k0 = kv0 + (size_t)keys[i] * D;
         double dot = 0.0;
-        for (int d = 0; d < D; ++d) dot += bf16_to_f64(q[d]) * bf16_to_f64(kr[d]);
+        for (int d = 0; d < D; ++d)
+            dot += elem(J->Q, q0 + d, J->fp8, J->q_descale) * elem(J->K, k0 + d, J->fp8, J->k_descale);
         s[i] = J->scale * dot;
         if (s[i] > m) m = s[i];
     }
@@ -202,8 +228,8 @@ static int attention_over_keys(const attn_job *J, int b, int h, int g, int r,
     for (int d = 0; d < D; ++d) o[d] = 0.0;
     for (int64_t i = 0; i < nk; ++i) {
         const double w = exp(s[i] - L);
-        const uint16_t *vr = Vbg + (size_t)keys[i] * D;
-        for (int d = 0; d < D; ++d) o[d] += w * bf16_to_f64(vr[d]);
+        const size_t v0 = kv0 + (size_t)keys[i] * D;
+        for (int d = 0; d < D; ++d) o[d] += w * elem(J->V, v0 + d, J->fp8, J->v_descale);
     }
     *lse = L;
     return ORACLE_OK;
@@ -239,7 +265,7 @@ static void *attn_worker(void *arg) {
  * dense reference (every block of the sequence's visible length).
  * Writes O (fp64, [n_rows, D]) and LSE (fp64, [n_rows]).
  */
-static int run_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+static int run_rows(const void *Q, const void *K, const void *V, int fp8, const double *descale,
                     const int32_t *tables, const int32_t *counts, const uint8_t *tile_mask,
                     int nQ, const int32_t *chunk_start, int B, int H_q, int H_kv, int C,
                     int L_max, int D, int blk, double scale, const int64_t *rows,
@@ -269,6 +295,10 @@ static int run_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
     for (int w = 0; w < n_threads; ++w) {
         attn_job *J = &jobs[w];
         J->Q = Q; J->K = K; J->V = V;
+        J->fp8 = fp8;
+        J->q_descale = fp8 ? descale[0] : 1.0;
+        J->k_descale = fp8 ? descale[1] : 1.0;
+        J->v_descale = fp8 ? descale[2] : 1.0;
         J->tables = tables; J->counts = counts; J->chunk_start = chunk_start;
         J->tile_mask = tile_mask; J->nQ = nQ;
         J->B = B; J->H_q = H_q; J->H_kv = H_kv; J->C = C; J->L_max = L_max;
@@ -307,8 +337,24 @@ int oracle_attention_rows(const uint16_t *Q, const uint16_t *K, const uint16_t *
                           const int32_t *chunk_start, int B, int H_q, int H_kv, int C,
                           int L_max, int D, int blk, double scale, const int64_t *rows,
                           int64_t n_rows, double *O, double *LSE, int n_threads) {
-    return run_rows(Q, K, V, tables, counts, NULL, 0, chunk_start, B, H_q, H_kv, C, L_max, D,
-                    blk, scale, rows, n_rows, O, LSE, n_threads);
+    return run_rows(Q, K, V, 0, NULL, tables, counts, NULL, 0, chunk_start, B, H_q, H_kv, C,
+                    L_max, D, blk, scale, rows, n_rows, O, LSE, n_threads);
+}
+
+/*
+ * The same attention on FP8 inputs: Q, K, V hold e4m3 codes and the real
+ * inputs are descale[0] * Q, descale[1] * K, descale[2] * V (per-tensor
+ * scale factors), each decoded exactly and then used in fp64 as above.
+ */
+int oracle_attention_rows_e4m3(const uint8_t *Q, const uint8_t *K, const uint8_t *V,
+                               const double *descale, const int32_t *tables,
+                               const int32_t *counts, const int32_t *chunk_start, int B, int H_q,
+                               int H_kv, int C, int L_max, int D, int blk, double scale,
+                               const int64_t *rows, int64_t n_rows, double *O, double *LSE,
+                               int n_threads) {
+    if (!descale) return ORACLE_EINVAL;
+    return run_rows(Q, K, V, 1, descale, tables, counts, NULL, 0, chunk_start, B, H_q, H_kv, C,
+                    L_max, D, blk, scale, rows, n_rows, O, LSE, n_threads);
 }
 
 /*
@@ -323,8 +369,8 @@ int oracle_attention_tile_rows(const uint16_t *Q, const uint16_t *K, const uint1
                                double scale, const int64_t *rows, int64_t n_rows, double *O,
                                double *LSE, int n_threads) {
     if (!mask) return ORACLE_EINVAL;
-    return run_rows(Q, K, V, NULL, NULL, mask, nQ, chunk_start, B, H_q, H_kv, C, L_max, D,
-                    blk, scale, rows, n_rows, O, LSE, n_threads);
+    return run_rows(Q, K, V, 0, NULL, NULL, NULL, mask, nQ, chunk_start, B, H_q, H_kv, C, L_max,
+                    D, blk, scale, rows, n_rows, O, LSE, n_threads);
 }
 
 /*

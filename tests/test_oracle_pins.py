@@ -513,3 +513,63 @@ def test_tile_span_tables_round_trip_and_order(span):
                     rebuilt[b, h, s * span + u, j[(bits >> u) & 1 == 1]] = True
     np.testing.assert_array_equal(rebuilt[:, :, :nQ], mask != 0)
     assert not rebuilt[:, :, nQ:].any()
+
+
+# ------------------------------------------------------------ FP8 (E4M3) inputs
+
+def test_e4m3_decode_matches_torch_on_every_code():
+    """The oracle's E4M3 decoder, written from the format's definition, against
+    torch's float8_e4m3fn conversion on all 256 codes (NaN codes included)."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = np.array([oracle.e4m3_decode(i) for i in range(256)])
+    assert np.array_equal(np.isnan(ref), np.isnan(mine))
+    np.testing.assert_array_equal(mine[~np.isnan(mine)], ref[~np.isnan(ref)])
+    assert mine[0x7E] == 448.0 and mine[0x01] == 2.0 ** -9 and mine[0x08] == 2.0 ** -6
+
+
+@pytest.mark.parametrize("cfg", [
+    # B, H_q, H_kv, D, blk, C, L_max, chunk_start
+    (1, 4, 1, 16, 8, 24, 64, (16,)),
+    (2, 4, 2, 32, 8, 16, 48, (32, 8)),
+])
+def test_e4m3_attention_equals_sdpa_on_dequantized_inputs(cfg):
+    """FP8 attention is the bf16 definition on the dequantized tensors: fp64
+    SDPA on descale * decode(codes) (decoded by torch), under the tables."""
+    B, H_q, H_kv, D, blk, C, L, cs = cfg
+    Q, K, V = _rand_qkv(sum(cfg[:7]) + 1, B, H_q, H_kv, C, L, D)
+    (q8, qd), (k8, kd), (v8, vd) = (workloads.quantize_e4m3(t) for t in (Q, K, V))
+    rng = np.random.default_rng(5)
+    mask = (rng.random((B, H_q, C // blk, L // blk)) < 0.5).astype(np.uint8)
+    mask[..., 0] = 1
+    T, cnt, _, _ = oracle.block_tables(mask, H_q // H_kv)
+    scale = 0.8 / math.sqrt(D)
+    O, LSE = oracle.attention_e4m3(q8, k8, v8, (qd, kd, vd), cs, blk, T, cnt, scale=scale)
+    deq = lambda c, d: (c.view(torch.float8_e4m3fn).to(torch.float64) * d)
+    Qd, Kd, Vd = deq(q8, qd), deq(k8, kd), deq(v8, vd)
+    # the union's key set, expanded to tokens, causal on top
+    allowed = torch.zeros(B, H_q, C, L, dtype=torch.bool)
+    for b in range(B):
+        for h in range(H_q):
+            sel = torch.zeros(L, dtype=torch.bool)
+            for j in T[b, h // (H_q // H_kv), :cnt[b, h // (H_q // H_kv)]]:
+                sel[j * blk:(j + 1) * blk] = True
+            allowed[b, h] = sel[None, :]
+    allowed &= _causal_allowed(B, H_q, C, L, cs)
+    Oref, LSEref = _sdpa_masked(Qd, Kd, Vd, allowed, scale)
+    np.testing.assert_allclose(O, Oref, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(LSE, LSEref, rtol=1e-10, atol=1e-10)
+
+
+def test_quantize_e4m3_round_trip_bound():
+    """The FP8 input encoding: |x - descale * decode(code)| is within half an
+    E4M3 step of x / descale (relative 2^-4 for normal codes, 2^-10 absolute
+    below 2^-6), and amax maps to 448."""
+    x = torch.randn(4096, generator=torch.Generator().manual_seed(3)) * 3
+    codes, d = workloads.quantize_e4m3(x)
+    dec = np.array([oracle.e4m3_decode(int(c)) for c in codes.numpy()])
+    y = x.double().numpy() / d
+    err = np.abs(dec - y)
+    bound = np.maximum(np.abs(y) * 2.0 ** -4, 2.0 ** -10)
+    assert np.all(err <= bound * (1 + 1e-12))
+    assert np.isclose(np.abs(dec).max(), 448.0)

@@ -47,6 +47,7 @@ __all__ = [
     "make_kv",
     "poison_beyond_kv_len",
     "pack_mask_bits",
+    "quantize_e4m3",
 ]
 
 
@@ -324,3 +325,15 @@ def pack_mask_bits(mask: np.ndarray) -> np.ndarray:
     padded[..., :nK] = mask != 0
     bytes_ = np.packbits(padded.reshape(B, H, nQ, nW, 4, 8), axis=-1, bitorder="little")
     return bytes_.reshape(B, H, nQ, nW, 4).copy().view("<u4").reshape(B, H, nQ, nW)
+
+
+def quantize_e4m3(x: torch.Tensor) -> Tuple[torch.Tensor, float]:
+    """FP8 E4M3 form of an input tensor for the FP8 path (an input encoding,
+    no method arithmetic): a per-tensor descale factor amax / 448 and the
+    codes of x / descale rounded to nearest by torch's float8_e4m3fn cast.
+    Returns (uint8 codes, descale)."""
+    xf = x.float()
+    amax = float(xf.abs().max())
+    descale = amax / 448.0 if amax > 0 else 1.0
+    codes = (xf / descale).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), descale
