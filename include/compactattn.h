@@ -176,6 +176,25 @@ int ca_paged_chunk_attention(const void *Q, const void *K, const void *V,
                              float *LSE, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * ca_chunk_attention on an FP8 (E4M3) cache. The pages use bf16; this is an
+ * extension for caches stored in 8 bits. Q8, K8, V8 hold E4M3 codes (one byte
+ * per element, same layouts as the bf16 tensors) and the attention inputs are
+ * q_descale * Q8, k_descale * K8, v_descale * V8 (per-tensor factors, > 0).
+ * Q.K^T and P.V run as E4M3 tensor-core products with fp32 accumulation; P
+ * is rounded to E4M3 as 2^(x + 8) with the running row max raised whenever a
+ * row max grows by more than 1/2, so it never saturates (P <= 2^8.5 < 448).
+ * O (bf16) and LSE (fp32) as ca_chunk_attention; tables == NULL (and counts
+ * == NULL) runs the dense path over every visible block. Supported: D = 128,
+ * blk in {64, 128}; other arguments and errors as ca_chunk_attention, plus
+ * CA_ERR_INVALID_ARG for a descale that is not a positive finite number.
+ */
+int ca_chunk_attention_fp8(const void *Q8, const void *K8, const void *V8, float q_descale,
+                           float k_descale, float v_descale, const int32_t *tables,
+                           const int32_t *counts, const int32_t *chunk_start, int B, int H_q,
+                           int H_kv, int C, int L_max, int D, int blk, float scale, void *O,
+                           float *LSE, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * The dense paged path (pages: the "dense attention baseline" the speedup is
  * quoted against): identical to ca_chunk_attention with
  * T_{b,g} = [0, ceil((chunk_start[b] + C) / blk)) for every group.

@@ -72,6 +72,7 @@ EXPORTED_SYMBOLS = (
     "ca_tile_span",
     "ca_build_kv_pages",
     "ca_build_block_tables_bits",
+    "ca_chunk_attention_fp8",
     "ca_paged_chunk_attention",
     "ca_build_tile_tables",
     "ca_tile_chunk_attention",
@@ -123,6 +124,9 @@ def load_library():
         lib.ca_compacted_chunk_attention.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P,
                                                      P, P, S, P]
         lib.ca_compacted_chunk_attention.restype = I
+        lib.ca_chunk_attention_fp8.argtypes = [P, P, P, F, F, F, P, P, P, I, I, I, I, I, I, I, F,
+                                               P, P, P, S, P]
+        lib.ca_chunk_attention_fp8.restype = I
         lib.ca_build_block_tables_bits.argtypes = [P, I, I, I, I, I, P, P, P, P, P]
         lib.ca_build_block_tables_bits.restype = I
         lib.ca_build_kv_pages.argtypes = [P, I, I, I, I, I, P, P, P, P, P]
@@ -585,4 +589,53 @@ def paged_chunk_attention(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
         B, H_q, H_kv, C, L_max, D, int(blk), float(scale), _ptr(O), _ptr(LSE), _ptr(workspace),
         workspace.numel(), _stream_handle(stream, Q.device))
     _check("ca_paged_chunk_attention", st)
+    return O, LSE
+
+
+# ------------------------------------------------------------- FP8 (E4M3) cache
+
+def chunk_attention_fp8(Q8: torch.Tensor, K8: torch.Tensor, V8: torch.Tensor,
+                        descale: Sequence[float], chunk_start: Sequence[int], blk: int,
+                        tables: Optional[torch.Tensor] = None,
+                        counts: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                        O: Optional[torch.Tensor] = None, LSE: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None,
+                        stream: Optional[torch.cuda.Stream] = None
+                        ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Chunk attention on E4M3 inputs (uint8 or float8_e4m3fn tensors with the
+    bf16 layouts; the real inputs are ``descale[i]`` times the codes). Tables
+    as in :func:`chunk_attention`, or none for the dense path. O is bf16."""
+    def codes(t, name, ndim):
+        if t.dtype == torch.float8_e4m3fn:
+            t = t.view(torch.uint8)
+        _need(t, name, torch.uint8, ndim)
+        return t
+    Q8, K8, V8 = codes(Q8, "Q8", 4), codes(K8, "K8", 4), codes(V8, "V8", 4)
+    B, H_q, C, D = Q8.shape
+    Bk, H_kv, L_max, Dk = K8.shape
+    if Bk != B or Dk != D or tuple(V8.shape) != tuple(K8.shape):
+        raise ValueError("shape mismatch")
+    if (tables is None) != (counts is None):
+        raise ValueError("give both tables and counts, or neither (dense path)")
+    if tables is not None:
+        _need(tables, "tables", torch.int32, 3)
+        _need(counts, "counts", torch.int32, 2)
+    dev = Q8.device
+    if O is None:
+        O = torch.empty((B, H_q, C, D), dtype=torch.bfloat16, device=dev)
+    _need(O, "O", torch.bfloat16, 4)
+    if LSE is None:
+        LSE = torch.empty((B, H_q, C), dtype=torch.float32, device=dev)
+    _need(LSE, "LSE", torch.float32, 3)
+    if workspace is None:
+        workspace = new_workspace(B, H_q, H_kv, C, blk, device=dev)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    qd, kd, vd = (float(x) for x in descale)
+    cs = _chunk_start_host(chunk_start, B)
+    st = load_library().ca_chunk_attention_fp8(
+        _ptr(Q8), _ptr(K8), _ptr(V8), qd, kd, vd, _ptr(tables), _ptr(counts), cs, B, H_q, H_kv,
+        C, L_max, D, int(blk), float(scale), _ptr(O), _ptr(LSE), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream, dev))
+    _check("ca_chunk_attention_fp8", st)
     return O, LSE

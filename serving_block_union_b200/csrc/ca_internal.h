@@ -41,6 +41,10 @@ struct AttnArgs {
     const int32_t *kv_indptr = nullptr;
     long long nnz = 0;
     const int32_t *chunk_len = nullptr;  // host [B], NULL: every chunk is C rows
+    // FP8 inputs: Q, K, V hold E4M3 codes; the real values are the codes times
+    // descale[0] (Q), descale[1] (K), descale[2] (V)
+    bool fp8 = false;
+    float descale[3] = {1.0f, 1.0f, 1.0f};
 };
 
 // Attention kernel modes: walk the tables over the cache in place; every block

@@ -151,6 +151,29 @@ int ca_paged_chunk_attention(const void *Q, const void *K, const void *V,
     return ca::launch_chunk_attention(a, ca::kModeTables, static_cast<cudaStream_t>(stream));
 }
 
+int ca_chunk_attention_fp8(const void *Q8, const void *K8, const void *V8, float q_descale,
+                           float k_descale, float v_descale, const int32_t *tables,
+                           const int32_t *counts, const int32_t *chunk_start, int B, int H_q,
+                           int H_kv, int C, int L_max, int D, int blk, float scale, void *O,
+                           float *LSE, void *workspace, size_t workspace_bytes, void *stream) {
+    const bool dense = tables == nullptr;
+    if (dense && counts) return CA_ERR_INVALID_ARG;
+    const int st = check_attention(Q8, K8, V8, tables, counts, dense, chunk_start, B, H_q, H_kv,
+                                   C, L_max, D, blk, scale, O, LSE, workspace, workspace_bytes);
+    if (st != CA_OK) return st;
+    for (float d : {q_descale, k_descale, v_descale})
+        if (!(d > 0.0f) || !isfinite(d)) return CA_ERR_INVALID_ARG;
+    if (D != 128) return CA_ERR_UNSUPPORTED;
+    ca::AttnArgs a{Q8, K8, V8, tables, counts, chunk_start, B, H_q, H_kv, C, L_max, D, blk,
+                   scale, O, LSE, workspace, workspace_bytes};
+    a.fp8 = true;
+    a.descale[0] = q_descale;
+    a.descale[1] = k_descale;
+    a.descale[2] = v_descale;
+    return ca::launch_chunk_attention(a, dense ? ca::kModeDense : ca::kModeTables,
+                                      static_cast<cudaStream_t>(stream));
+}
+
 int ca_chunk_attention(const void *Q, const void *K, const void *V, const int32_t *tables,
                        const int32_t *counts, const int32_t *chunk_start, int B, int H_q,
                        int H_kv, int C, int L_max, int D, int blk, float scale, void *O,

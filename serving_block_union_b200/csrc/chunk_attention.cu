@@ -124,6 +124,7 @@ struct Params {
     float *part_lse;              // [n_rest][split][256] base-2 LSE of a segment's rows
     float *part_o;                // [n_rest][split][256][D] normalised partial O
     float scale_log2;
+    float o_scale;              // factor on O (the V descale of FP8 inputs, else 1)
     const int32_t *tables;      // or, in the paged form, kv_indices (global pages)
     const int32_t *counts;
     const int32_t *kv_indptr;   // paged form: rows of (b, g) in kv_indices; else NULL
@@ -136,10 +137,11 @@ struct Params {
     unsigned char b_order[kMaxBatch];
 };
 
-template <int D, int BLK>
+template <int D, int BLK, bool F8 = false>
 struct Layout {
-    static constexpr int kQTile = kTileM * D * 2;  // D/64 sub-tiles of 128 rows x 128 B
-    static constexpr int kKV = BLK * D * 2;        // D/64 sub-tiles of BLK rows x 128 B
+    static constexpr int kEB = F8 ? 1 : 2;           // bytes per Q / K / V element
+    static constexpr int kQTile = kTileM * D * kEB;  // D*kEB/128 sub-tiles of 128 rows x 128 B
+    static constexpr int kKV = BLK * D * kEB;        // D*kEB/128 sub-tiles of BLK rows x 128 B
     // P tile (shared-memory P only): BLK/64 sub-tiles of 128 rows x 128 B
     static constexpr int kPTile = kPSmem ? kTileM * BLK * 2 : 0;
     static constexpr int kXchBytes = kColSplit == 2 ? 2 * 4 * 2 * 32 * 4 : 0;
@@ -167,6 +169,7 @@ struct Layout {
     static_assert(kPSmem || kStagesV >= 2, "need two V stages");
     static_assert(!kPSmem || kPChunkKeys == 64, "shared-memory P hands over 64-key sub-tiles");
     static_assert(kDynamic <= kSmemBudget, "shared memory budget exceeded");
+    static_assert(!F8 || !kPSmem, "FP8 keeps P in TMEM");
 };
 
 // KV block index of a table entry (span-table entries carry Q-block bits
@@ -239,21 +242,34 @@ __device__ __forceinline__ void tmem_ld_row<32>(uint32_t taddr, uint32_t (&r)[32
     tmem_ld32(taddr, r);
 }
 
-template <int D, int BLK, int MODE>
+template <int D, int BLK, int MODE, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params P) {
-    using L = Layout<D, BLK>;
+    using L = Layout<D, BLK, F8>;
     constexpr bool DENSE = MODE == kModeDense;
     constexpr bool COMPACT = MODE == kModeCompact;  // K/V block t sits at row t * BLK
     constexpr bool PERTILE = MODE == kModePerTile;  // one head per tile, span tables
     constexpr int NST = L::kStages;
     constexpr int NSK = L::kStagesK;  // K ring
     constexpr int NSV = L::kStagesV;  // V ring
-    constexpr int DCH = D / 64;  // 64-element (128-byte) sub-tiles along D
-    constexpr uint32_t kIdescS = idesc_bf16_f32(kTileM, BLK, false);
-    constexpr uint32_t kIdescPV = idesc_bf16_f32(kTileM, D, true);
+    // FP8 (E4M3 Q, K, V; kind::f8f6f4 MMAs; P rounded to E4M3 in TMEM)
+    constexpr int EB = L::kEB;
+    constexpr int DCH = D * EB / 128;  // 128-byte sub-tiles along D
+    constexpr int XIN = 128 / EB;      // elements in a 128-byte sub-tile row
+    constexpr int KS = 32 / EB;        // elements per MMA K step (32 bytes)
+    constexpr uint32_t kIdescS =
+        F8 ? idesc_e4m3_f32(kTileM, BLK, false) : idesc_bf16_f32(kTileM, BLK, false);
+    constexpr uint32_t kIdescPV =
+        F8 ? idesc_e4m3_f32(kTileM, D, true) : idesc_bf16_f32(kTileM, D, true);
+    // FP8 P is 2^(x + 8) with the running max raised whenever a row max grows
+    // by more than 1/2, so P <= 2^8.5 fits E4M3 (max 448) and values down to
+    // 2^-17 of the row max stay representable; bf16 P is 2^x, threshold 8.
+    constexpr float kThresh = F8 ? 0.5f : kRescaleThreshold;
+    constexpr float kPBias = F8 ? 8.0f : 0.0f;
+    static_assert(!F8 || MODE == kModeTables || MODE == kModeDense,
+                  "FP8 runs the table and dense paths");
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -402,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int t = 0; t < 2; ++t)
                     for (int dc = 0; dc < DCH; ++dc)
                         tma_load_3d(smem + L::kQOff + t * L::kQTile + dc * (kTileM * 128), &tmQ,
-                                    q_full, dc * 64, r0 + t * R, b * P.H_q + head0);
+                                    q_full, dc * XIN, r0 + t * R, b * P.H_q + head0);
             }
             q_issued = true;
             // K(j) into ring stage j % NSK, V(j) into j % NSV (lane 0 only);
@@ -413,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive_expect_tx(k_full + s, L::kKV);
                 for (int dc = 0; dc < DCH; ++dc)
                     tma_load_3d(smem + L::kKOff + s * L::kKV + dc * (BLK * 128), &tmK,
-                                k_full + s, dc * 64, blk_idx * BLK, b * P.H_kv + g);
+                                k_full + s, dc * XIN, blk_idx * BLK, b * P.H_kv + g);
                 k_issued = j + 1;
                 return true;
             };
@@ -423,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive_expect_tx(v_full + s, L::kKV);
                 for (int dc = 0; dc < DCH; ++dc)
                     tma_load_3d(smem + L::kVOff + s * L::kKV + dc * (BLK * 128), &tmV,
-                                v_full + s, dc * 64, blk_idx * BLK, b * P.H_kv + g);
+                                v_full + s, dc * XIN, blk_idx * BLK, b * P.H_kv + g);
                 v_issued = j + 1;
                 return true;
             };
@@ -497,13 +513,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t a0 = q_lo + t * (L::kQTile >> 4);
                 const uint32_t b0 = k_lo + slot * kStageUnits;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    // 16 bf16 = 32 B steps inside a 128-B swizzle row; a new 64-column
-                    // sub-tile every 4 steps
+                for (int kk = 0; kk < D / KS; ++kk) {
+                    // 32-byte K steps (16 bf16 / 32 E4M3) inside a 128-B swizzle
+                    // row; a new 128-byte sub-tile every 4 steps
                     const uint32_t ao = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
                     const uint32_t bo = ((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4;
-                    mma_ss_w(tmem + t * 128, a0 + ao, q_hi, b0 + bo, k_hi, kIdescS,
-                             kk > 0 ? 1u : 0u);
+                    if constexpr (F8)
+                        mma_ss_w8(tmem + t * 128, a0 + ao, q_hi, b0 + bo, k_hi, kIdescS,
+                                  kk > 0 ? 1u : 0u);
+                    else
+                        mma_ss_w(tmem + t * 128, a0 + ao, q_hi, b0 + bo, k_hi, kIdescS,
+                                 kk > 0 ? 1u : 0u);
                 }
             };
             // P.V of tile t, chunk by chunk as the softmax hands P over; false if a
@@ -514,12 +534,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < NPC; ++c) {
                     if (!mbar_wait(p_full + t * NPC + c, par, ab)) return false;
                     tc_fence_after();
-                    constexpr int KPC = L::kPChunkKeys / 16;  // MMAs (K = 16) per chunk
+                    constexpr int KPC = L::kPChunkKeys / KS;  // MMAs (one K step each) per chunk
 #pragma unroll
                     for (int kk = KPC * c; kk < KPC * c + KPC; ++kk) {
-                        mma_ts_w(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
-                                 b0 + ((kk * (16 * 128)) >> 4), v_hi, kIdescPV,
-                                 (acc || kk > 0) ? 1u : 0u);
+                        // a K step is 8 TMEM columns of P (2 bf16 or 4 E4M3 per
+                        // column) and KS rows of V (128 bytes per row)
+                        if constexpr (F8)
+                            mma_ts_w8(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                                      b0 + ((kk * (KS * 128)) >> 4), v_hi, kIdescPV,
+                                      (acc || kk > 0) ? 1u : 0u);
+                        else
+                            mma_ts_w(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                                     b0 + ((kk * (KS * 128)) >> 4), v_hi, kIdescPV,
+                                     (acc || kk > 0) ? 1u : 0u);
                     }
                 }
                 return true;
@@ -656,6 +683,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
 
         float m_run = -INFINITY, l_run = 0.0f;  // l_run: this warp's columns only
+        float lh_run = 0.0f;  // FP8: the same sum over the E4M3-rounded P
         bool ok = true;
         for (int j = 0; j < n_run; ++j) {
             ok = mbar_wait(s_full + t, j & 1, ab);
@@ -754,7 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float m_blk = pmax * sl2;
             const float m_new = fmaxf(m_run, m_blk);
             const bool old_finite = m_run != -INFINITY;
-            const bool upd = old_finite ? (m_new > m_run + kRescaleThreshold)
+            const bool upd = old_finite ? (m_new > m_run + kThresh)
                                         : (m_new != -INFINITY);
             float alpha = 1.0f;
             if (upd) {
@@ -785,15 +813,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             // row sum in four f32x2 accumulators; the MUFU unit does most pairs,
             // the FMA pipe the pairs use_poly_pair() selects
             const uint64_t sl2x2 = f2_pack(sl2, sl2);
-            const uint64_t nm2 = f2_pack(-m_use, -m_use);
+            const uint64_t nm2 = f2_pack(kPBias - m_use, kPBias - m_use);
             uint64_t acc2[4];
+            uint64_t acch[2] = {0ull, 0ull};  // FP8: sums of the rounded P
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc2[k] = 0ull;
 #pragma unroll
             for (int cl = 0; cl < CPW; ++cl) {
                 constexpr int CK = L::kPChunkKeys;
                 const int c = hf * CPW + cl;  // P chunk index within the row
-                uint32_t pk[CK / 2];
+                constexpr int PCOLS = CK * EB / 4;  // TMEM columns of a P chunk
+                uint32_t pk[CK / 2];  // bf16 pairs; FP8: E4M3 quads in pk[0, CK/4)
+                uint64_t p_prev = 0ull;
 #pragma unroll
                 for (int i = 0; i < CK / 2; ++i) {
                     const int e0 = cl * CK + 2 * i;  // element in this warp's s[]
@@ -801,8 +832,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t p2 = use_poly_pair(c * CK / 2 + i)
                                             ? exp2_poly2(x2)
                                             : f2_pack(ex2_approx(f2_lo(x2)), ex2_approx(f2_hi(x2)));
-                    acc2[i & 3] = f2_add(acc2[i & 3], p2);
-                    pk[i] = pack_bf16x2(f2_lo(p2), f2_hi(p2));
+                    if constexpr (F8) {
+                        // O is normalised by the sum of the E4M3 values P.V uses
+                        // (an exact convex combination of V rows); the LSE keeps
+                        // the fp32 sum
+                        acc2[i & 3] = f2_add(acc2[i & 3], p2);
+                        if (i & 1) {
+                            const uint32_t q4 = pack_e4m3x4(f2_lo(p_prev), f2_hi(p_prev),
+                                                            f2_lo(p2), f2_hi(p2));
+                            pk[i >> 1] = q4;
+                            acch[(i >> 1) & 1] = f2_add(
+                                acch[(i >> 1) & 1],
+                                f2_add(e4m3x2_to_f32x2(static_cast<uint16_t>(q4)),
+                                       e4m3x2_to_f32x2(static_cast<uint16_t>(q4 >> 16))));
+                        } else {
+                            p_prev = p2;
+                        }
+                    } else {
+                        acc2[i & 3] = f2_add(acc2[i & 3], p2);
+                        pk[i] = pack_bf16x2(f2_lo(p2), f2_hi(p2));
+                    }
                 }
                 if constexpr (kPSmem) {
                     if (cl == 0 && j > 0) {
@@ -834,8 +883,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_arrive_lane0(p_full + t * NPC + c, lane);
                 } else {
 #pragma unroll
-                    for (int q = 0; q < CK / 32; ++q)
-                        tmem_st16(tS + c * (CK / 2) + q * 16, pk + q * 16);
+                    for (int q = 0; q < PCOLS / 16; ++q)
+                        tmem_st16(tS + c * PCOLS + q * 16, pk + q * 16);
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
@@ -846,6 +895,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             acc2[0] = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
             const float sum = f2_lo(acc2[0]) + f2_hi(acc2[0]);
             l_run += sum;
+            if constexpr (F8) {
+                acch[0] = f2_add(acch[0], acch[1]);
+                lh_run = lh_run * alpha + (f2_lo(acch[0]) + f2_hi(acch[0]));
+            }
         }
         bool have_o = false;
         if (n_run > 0 && __all_sync(0xffffffffu, ok)) {
@@ -861,8 +914,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 have_o = false;
             }
         }
-        const float inv_l = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-        const float lse2 = (l_run > 0.0f && have_o) ? m_run + log2f(l_run) : -INFINITY;
+        const float l_o = F8 ? lh_run : l_run;  // the sum O is normalised by
+        const float inv_l = l_o > 0.0f ? P.o_scale / l_o : 0.0f;
+        const float lse2 = (l_run > 0.0f && have_o) ? m_run + log2f(l_run) - kPBias : -INFINITY;
         uint16_t *orow = P.O + (((size_t)b * P.H_q + h) * P.C + r) * D + hf * DW;
         float *lse_out = (valid && hf == 0 && P.LSE != nullptr)
                              ? P.LSE + ((size_t)b * P.H_q + h) * P.C + r
@@ -998,24 +1052,28 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-bool encode_3d(CUtensorMap *map, const void *base, uint64_t d0, uint64_t d1, uint64_t d2,
-               uint32_t b0, uint32_t b1, uint32_t b2) {
+// 3-D tiled map over a contiguous [d2][d1][d0] tensor of bf16 (eb = 2) or
+// 8-bit (eb = 1, E4M3 codes moved as bytes) elements, 128-byte swizzle.
+bool encode_3d(CUtensorMap *map, const void *base, int eb, uint64_t d0, uint64_t d1,
+               uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {d0, d1, d2};
-    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint64_t strides[2] = {d0 * eb, d0 * d1 * eb};
     cuuint32_t box[3] = {b0, b1, b2};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
+    const CUtensorMapDataType dt =
+        eb == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = fn(map, dt, 3, const_cast<void *>(base), dims,
                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int BLK, int MODE>
+template <int D, int BLK, int MODE, bool F8 = false>
 int launch_t(const AttnArgs &a, cudaStream_t stream) {
-    using L = Layout<D, BLK>;
-    auto kern = chunk_attn_kernel<D, BLK, MODE>;
+    using L = Layout<D, BLK, F8>;
+    auto kern = chunk_attn_kernel<D, BLK, MODE, F8>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -1040,10 +1098,15 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
     const int n_tiles = (a.C + R - 1) / R;
     const int n_pairs = (n_tiles + 1) / 2;
 
+    constexpr int EB = L::kEB;
+    constexpr uint32_t XIN = 128 / EB;  // box width: one 128-byte swizzle row
     CUtensorMap tq, tk, tv;
-    if (!encode_3d(&tq, a.Q, (uint64_t)D, (uint64_t)a.C, (uint64_t)a.B * a.H_q, 64, R, pack) ||
-        !encode_3d(&tk, a.K, (uint64_t)D, (uint64_t)a.L_max, (uint64_t)a.B * a.H_kv, 64, BLK, 1) ||
-        !encode_3d(&tv, a.V, (uint64_t)D, (uint64_t)a.L_max, (uint64_t)a.B * a.H_kv, 64, BLK, 1))
+    if (!encode_3d(&tq, a.Q, EB, (uint64_t)D, (uint64_t)a.C, (uint64_t)a.B * a.H_q, XIN, R,
+                   pack) ||
+        !encode_3d(&tk, a.K, EB, (uint64_t)D, (uint64_t)a.L_max, (uint64_t)a.B * a.H_kv, XIN, BLK,
+                   1) ||
+        !encode_3d(&tv, a.V, EB, (uint64_t)D, (uint64_t)a.L_max, (uint64_t)a.B * a.H_kv, XIN, BLK,
+                   1))
         return CA_ERR_CUDA;
 
     Params P;
@@ -1056,7 +1119,8 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
     P.R = R;
     P.n_pairs = n_pairs;
     P.nKVmax = a.L_max / BLK;
-    P.scale_log2 = a.scale * 1.4426950408889634f;
+    P.scale_log2 = a.scale * 1.4426950408889634f * (F8 ? a.descale[0] * a.descale[1] : 1.0f);
+    P.o_scale = F8 ? a.descale[2] : 1.0f;
     P.tables = a.tables;
     P.counts = a.counts;
     P.kv_indptr = a.kv_indptr;
@@ -1128,6 +1192,17 @@ int current_sm_count() {
 }
 
 int launch_chunk_attention(const AttnArgs &a, int mode, cudaStream_t stream) {
+    if (a.fp8) {
+        if (a.D != 128 || (mode != kModeTables && mode != kModeDense)) return CA_ERR_UNSUPPORTED;
+        const bool dense = mode == kModeDense;
+        if (a.blk == 128)
+            return dense ? launch_t<128, 128, kModeDense, true>(a, stream)
+                         : launch_t<128, 128, kModeTables, true>(a, stream);
+        if (a.blk == 64)
+            return dense ? launch_t<128, 64, kModeDense, true>(a, stream)
+                         : launch_t<128, 64, kModeTables, true>(a, stream);
+        return CA_ERR_UNSUPPORTED;
+    }
 #define CA_DISPATCH(D_, BLK_)                                                         \
     if (a.D == D_ && a.blk == BLK_) {                                                 \
         if (mode == kModeDense) return launch_t<D_, BLK_, kModeDense>(a, stream);     \
