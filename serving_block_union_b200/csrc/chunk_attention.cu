@@ -114,6 +114,13 @@ constexpr int kPChunkKeysCfg = CA_P_CHUNK_KEYS;
 #endif
 constexpr bool kPSmem = CA_P_SMEM != 0;
 static_assert(!kPSmem || kColSplit == 1, "P in shared memory needs one softmax warp per row");
+
+// S(j+1) in two N = 64 halves (128-key blocks, P in TMEM): P occupies the
+// first 64 columns of S only, so the upper half (keys 64..127) is computed as
+// soon as the softmax has loaded S(j); only the lower half waits for P.V(j).
+#ifndef CA_SPLIT_S
+#define CA_SPLIT_S 0
+#endif
 static_assert(kPChunkKeysCfg == 32 || kPChunkKeysCfg == 64 || kPChunkKeysCfg == 128,
               "P chunk must be 32, 64 or 128 keys");
 
@@ -266,6 +273,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // FP8 P is 2^(x + 8) with the running max raised whenever a row max grows
     // by more than 1/2, so P <= 2^8.5 fits E4M3 (max 448) and values down to
     // 2^-17 of the row max stay representable; bf16 P is 2^x, threshold 8.
+    constexpr bool kSplitS = CA_SPLIT_S != 0 && !kPSmem && BLK == 128 && kColSplit == 1;
+    constexpr uint32_t kIdescS64 =
+        F8 ? idesc_e4m3_f32(kTileM, 64, false) : idesc_bf16_f32(kTileM, 64, false);
     constexpr float kThresh = F8 ? 0.5f : kRescaleThreshold;
     constexpr float kPBias = F8 ? 8.0f : 0.0f;
     static_assert(!F8 || MODE == kModeTables || MODE == kModeDense,
@@ -526,6 +536,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  kk > 0 ? 1u : 0u);
                 }
             };
+            // one N = 64 half of S(t): keys 64h .. 64h + 63 of the block (rows
+            // 64h.. of every K sub-tile) into TMEM columns 64h ..
+            auto issue_s_half = [&](int t, int slot, int h) {
+                const uint32_t a0 = q_lo + t * (L::kQTile >> 4);
+                const uint32_t b0 = k_lo + slot * kStageUnits + ((h * 64 * 128) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / KS; ++kk) {
+                    const uint32_t ao = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
+                    const uint32_t bo = ((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4;
+                    if constexpr (F8)
+                        mma_ss_w8(tmem + t * 128 + h * 64, a0 + ao, q_hi, b0 + bo, k_hi,
+                                  kIdescS64, kk > 0 ? 1u : 0u);
+                    else
+                        mma_ss_w(tmem + t * 128 + h * 64, a0 + ao, q_hi, b0 + bo, k_hi,
+                                 kIdescS64, kk > 0 ? 1u : 0u);
+                }
+            };
             // P.V of tile t, chunk by chunk as the softmax hands P over; false if a
             // wait gave up.
             auto issue_pv = [&](int t, int slot, bool acc, uint32_t par) -> bool {
@@ -608,7 +635,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!more) tc_commit(o_full + 1);
                 tc_commit(v_empty + vs);
             }
-            for (int j = 0; !kPSmem && j < n_run && ok; ++j) {
+            // Split S: per tile, S_hi(j + 1) once the softmax has loaded S(j),
+            // then P.V(j), then S_lo(j + 1) (which overwrites P's columns; the
+            // tensor core runs one CTA's MMAs in issue order).
+            for (int j = 0; kSplitS && j < n_run && ok; ++j) {
+                const int s = j % NST;
+                const bool more = j + 1 < n_run;
+                const int s1 = (j + 1) % NST;
+                if (!(ok = mbar_wait(v_full + s, (j / NST) & 1, ab))) break;
+                if (more && !(ok = mbar_wait(k_full + s1, ((j + 1) / NST) & 1, ab))) break;
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (more) {
+                        if (!(ok = mbar_wait(s_free + t, j & 1, ab))) break;
+                        tc_fence_after();
+                        issue_s_half(t, s1, 1);
+                    }
+                    if (!(ok = issue_pv(t, s, j > 0, j & 1))) break;
+                    if (t == 1) tc_commit(v_empty + s);
+                    if (more) {
+                        issue_s_half(t, s1, 0);
+                        tc_commit(s_full + t);
+                        if (t == 1) tc_commit(k_empty + s1);
+                    } else {
+                        tc_commit(o_full + t);
+                    }
+                }
+            }
+            for (int j = 0; !kPSmem && !kSplitS && j < n_run && ok; ++j) {
                 const int s = j % NST;
                 const uint32_t ph = (j / NST) & 1;
                 const bool more = j + 1 < n_run;
@@ -721,6 +775,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_arrive_lane0(p_full + t * NPC + c, lane);
                     }
                 } else {
+                    if constexpr (kSplitS) {
+                        // S(j) is not needed: its upper half can take S(j + 1)
+                        tc_fence_before();
+                        __syncwarp();
+                        mbar_arrive_lane0(s_free + t, lane);
+                    }
 #pragma unroll
                     for (int cl = 0; cl < CPW; ++cl) {
                         constexpr int CK = L::kPChunkKeys;
@@ -743,7 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int i = 0; i < CW; ++i) s[i] = __uint_as_float(v[i]);
             }
-            if constexpr (kPSmem) {
+            if constexpr (kPSmem || kSplitS) {
                 // S(j) is in registers: its TMEM columns can take S(j + 1)
                 tc_fence_before();
                 __syncwarp();
