@@ -44,11 +44,17 @@ KERNEL_SOURCES = [os.path.join(ROOT, "serving_block_union_b200", "csrc", f)
 
 
 def kernel_source_hash() -> str:
+    """Hash of the attention kernel's code (comments and whitespace removed, so
+    that a documentation edit does not invalidate a profile of the same code)."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -20,7 +20,17 @@
 // same time: they walk its blocks in lockstep, each block comes from HBM once
 // and then from L2. (A persistent stream-K schedule that balances the last
 // wave staggers the CTAs instead and read several times more DRAM; under the
-// 1 kW power cap that sustained runs reach, it was not faster either.)
+// 1 kW power cap that sustained runs reach, it was not faster either.) When
+// the items do not fill the SMs evenly, the items past the last full wave are
+// cut into segments of their block lists (split-KV): each segment CTA writes a
+// normalised partial O and its LSE to the workspace and the item's last CTA
+// merges them (an atomic counter, no waiting).
+//
+// FP8 (template flag): E4M3 Q, K, V, kind::f8f6f4 MMAs (K = 32 per step), P
+// rounded to E4M3 as 2^(x + 8) in TMEM (four values per column). Two build
+// switches keep measured alternatives that were slower: P in shared memory
+// (CA_P_SMEM) and S in two N = 64 halves (CA_SPLIT_S); both add shared-memory
+// traffic to MMAs that already use all of its bandwidth.
 //
 // Warp roles (384 threads, one CTA per SM):
 //   warps 0-3  softmax + epilogue of tile 0 (thread = TMEM lane = packed row)
