@@ -232,7 +232,7 @@ def run_reference(args, wl, name=None):
     mask = workloads.make_mask(wl)
     Q, K, V = workloads.make_qkv(wl)
     vals, rows_used, secs, threads = [], 0, 0.0, 1
-    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    per_step = max(0.5, 60.0 / max(1, args.steps + args.warmup))
     for i in range(args.warmup + args.steps):
         v, n, dt, threads = oracle_sample_rate(wl, mask, Q, K, V, target_s=per_step, seed=i)
         if i >= args.warmup:
