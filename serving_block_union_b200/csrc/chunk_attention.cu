@@ -125,6 +125,18 @@ constexpr int kPChunkKeysCfg = CA_P_CHUNK_KEYS;
 constexpr bool kPSmem = CA_P_SMEM != 0;
 static_assert(!kPSmem || kColSplit == 1, "P in shared memory needs one softmax warp per row");
 
+// Exponentials before the row max (bf16, P in TMEM): after the first block the
+// softmax starts the exponentials of block j with the running max of the
+// earlier blocks as reference and computes the block's max alongside; a max
+// that grew past the rescale threshold is taken into account for the next
+// blocks (O is rescaled before P(j+1) lands, the row sum at once). A block
+// whose max jumps by more than 2^kEarlyGuard takes the max-first path, so P
+// stays finite.
+#ifndef CA_EARLY_EXP
+#define CA_EARLY_EXP 0
+#endif
+constexpr float kEarlyGuard = 64.0f;
+
 // S(j+1) in two N = 64 halves (128-key blocks, P in TMEM): P occupies the
 // first 64 columns of S only, so the upper half (keys 64..127) is computed as
 // soon as the softmax has loaded S(j); only the lower half waits for P.V(j).
@@ -284,6 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // by more than 1/2, so P <= 2^8.5 fits E4M3 (max 448) and values down to
     // 2^-17 of the row max stay representable; bf16 P is 2^x, threshold 8.
     constexpr bool kSplitS = CA_SPLIT_S != 0 && !kPSmem && BLK == 128 && kColSplit == 1;
+    constexpr bool kEarly = CA_EARLY_EXP != 0 && !F8 && !kPSmem && kColSplit == 1;
     constexpr uint32_t kIdescS64 =
         F8 ? idesc_e4m3_f32(kTileM, 64, false) : idesc_bf16_f32(kTileM, 64, false);
     constexpr float kThresh = F8 ? 0.5f : kRescaleThreshold;
@@ -747,6 +760,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
 
         float m_run = -INFINITY, l_run = 0.0f;  // l_run: this warp's columns only
+        float pend = 1.0f;  // O rescale still owed (exponentials-first blocks)
         float lh_run = 0.0f;  // FP8: the same sum over the E4M3-rounded P
         bool ok = true;
         for (int j = 0; j < n_run; ++j) {
@@ -828,19 +842,92 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (c > lim) s[c] = -INFINITY;
             }
             // row max: 8 independent chains of 3-input max, then a short tree
-            float mx8[8];
+            auto row_max = [&]() -> float {
+                float mx8[8];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+                for (int k = 0; k < 8; ++k) mx8[k] = s[k];
 #pragma unroll
-            for (int c = 8; c + 8 < CW; c += 16)
+                for (int c = 8; c + 8 < CW; c += 16)
 #pragma unroll
-                for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], s[c + k], s[c + 8 + k]);
-            if ((CW - 8) % 16 != 0) {
+                    for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], s[c + k], s[c + 8 + k]);
+                if ((CW - 8) % 16 != 0) {
 #pragma unroll
-                for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], s[CW - 8 + k]);
+                    for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], s[CW - 8 + k]);
+                }
+                return fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
+                             fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
+            };
+            // exponentials of P chunk cl with reference m (bf16 pairs into pk, row
+            // sum into acc2)
+            auto exp_chunk = [&](int cl, float m_ref, uint32_t(&pk)[L::kPChunkKeys / 2],
+                                 uint64_t(&acc2)[4]) {
+                constexpr int CK = L::kPChunkKeys;
+                const uint64_t sl2x2 = f2_pack(sl2, sl2);
+                const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
+#pragma unroll
+                for (int i = 0; i < CK / 2; ++i) {
+                    const int e0 = cl * CK + 2 * i;
+                    const uint64_t x2 = f2_fma(f2_pack(s[e0], s[e0 + 1]), sl2x2, nm2);
+                    const uint64_t p2 = f2_pack(ex2_approx(f2_lo(x2)), ex2_approx(f2_hi(x2)));
+                    acc2[i & 3] = f2_add(acc2[i & 3], p2);
+                    pk[i] = pack_bf16x2(f2_lo(p2), f2_hi(p2));
+                }
+            };
+            // hands P chunk c (in pk) to the P.V MMA through TMEM
+            auto hand_over = [&](int c, const uint32_t(&pk)[L::kPChunkKeys / 2]) {
+                constexpr int PCOLS = L::kPChunkKeys * EB / 4;
+#pragma unroll
+                for (int q = 0; q < PCOLS / 16; ++q)
+                    tmem_st16(tS + c * PCOLS + q * 16, pk + q * 16);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                mbar_arrive_lane0(p_full + t * NPC + c, lane);
+            };
+            // O *= a on the rows where a != 1 (O holds P.V up to block j - 1:
+            // S(j) was committed after that P.V was issued)
+            auto rescale_o = [&](float a) {
+#pragma unroll
+                for (int c = 0; c < DW / 16; ++c) {
+                    uint32_t v[16];
+                    tmem_ld16(tO + c * 16, v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
+                    tmem_st16(tO + c * 16, v);
+                }
+            };
+            if constexpr (kEarly) {
+                if (__all_sync(0xffffffffu, m_run != -INFINITY)) {
+                    // exponentials first, with the running max as reference
+                    const float m_ref = m_run;
+                    uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+                    uint32_t pk0[L::kPChunkKeys / 2];
+                    exp_chunk(0, m_ref, pk0, acc2);
+                    const float m_blk = row_max() * sl2;
+                    if (!__any_sync(0xffffffffu, m_blk > m_ref + kEarlyGuard)) {
+                        if (__any_sync(0xffffffffu, pend != 1.0f)) rescale_o(pend);
+                        pend = 1.0f;
+                        hand_over(0, pk0);
+#pragma unroll
+                        for (int cl = 1; cl < NPC; ++cl) {
+                            uint32_t pk[L::kPChunkKeys / 2];
+                            exp_chunk(cl, m_ref, pk, acc2);
+                            hand_over(cl, pk);
+                        }
+                        acc2[0] = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
+                        l_run += f2_lo(acc2[0]) + f2_hi(acc2[0]);
+                        if (m_blk > m_ref + kThresh) {  // raise the max for later blocks
+                            const float a = ex2_approx(m_ref - m_blk);
+                            l_run *= a;
+                            m_run = m_blk;
+                            pend = a;
+                        }
+                        continue;
+                    }
+                    // a jump past the guard: the max-first path below
+                }
             }
-            float pmax = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
-                               fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
+            float pmax = row_max();
             if (kColSplit == 2) {
                 float other;
                 if (!exchange(pmax, other)) {
@@ -865,18 +952,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // DW columns of O.
             const bool need = upd && old_finite && j > 0;
             // (with P in shared memory the rescale waits for P.V(j - 1) first; it
-            // runs inside the chunk loop below)
-            if (!kPSmem && __any_sync(0xffffffffu, need)) {
-                const float a = need ? alpha : 1.0f;
-#pragma unroll
-                for (int c = 0; c < DW / 16; ++c) {
-                    uint32_t v[16];
-                    tmem_ld16(tO + c * 16, v);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
-                    tmem_st16(tO + c * 16, v);
-                }
+            // runs inside the chunk loop below). A rescale still owed by an
+            // exponentials-first block is folded in.
+            if (!kPSmem && __any_sync(0xffffffffu, need || pend != 1.0f)) {
+                rescale_o((need ? alpha : 1.0f) * pend);
             }
+            pend = 1.0f;
             const float m_use = m_run == -INFINITY ? 0.0f : m_run;
             l_run *= alpha;
             // exponentials in pairs: x = s * scale_log2 - m as one f32x2 FMA, the
@@ -985,7 +1066,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         const float l_o = F8 ? lh_run : l_run;  // the sum O is normalised by
-        const float inv_l = l_o > 0.0f ? P.o_scale / l_o : 0.0f;
+        // (pend: the last block's O rescale, owed if it raised the max)
+        const float inv_l = l_o > 0.0f ? P.o_scale * pend / l_o : 0.0f;
         const float lse2 = (l_run > 0.0f && have_o) ? m_run + log2f(l_run) - kPBias : -INFINITY;
         uint16_t *orow = P.O + (((size_t)b * P.H_q + h) * P.C + r) * D + hf * DW;
         float *lse_out = (valid && hf == 0 && P.LSE != nullptr)
