@@ -428,19 +428,22 @@ def run_ours(args, chunks):
             dist.barrier(device_ids=[local])
         torch.cuda.synchronize(dev)
 
-    def timed(fn, steps, warm):
+    def timed_round_robin(fns, steps, warm):
         for _ in range(warm):
-            fn()
+            for fn in fns:
+                fn()
         barrier()
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(steps)]
-        for a, b in ev:
-            flush.zero_()
-            a.record(stream)
-            fn()
-            b.record(stream)
+        ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)] for _ in fns]
+        for i in range(steps):
+            for f, fn in enumerate(fns):
+                a, b = ev[f][i]
+                flush.zero_()
+                a.record(stream)
+                fn()
+                b.record(stream)
         barrier()
-        return [a.elapsed_time(b) for a, b in ev]
+        return [[a.elapsed_time(b) for a, b in ev[f]] for f in range(len(fns))]
 
     # work count of one step (from the step's own tables)
     build()
@@ -488,19 +491,15 @@ def run_ours(args, chunks):
         return g.replay
 
     step_run, attn_run, dense_run = graphed(step), graphed(attend), graphed(dense)
+    # Every path is timed in each step, round robin, so that all of them see
+    # the same clocks and power state (a path timed alone in its own loop gets
+    # whatever the loops before it left: the 1 kW power cap lowers the clocks
+    # as the run heats up). build_bits rewrites the tables the FP8 runs read.
     with ClockSampler(gpu_index) as clk:
-        step_ms = timed(step_run, args.steps, args.warmup)
-        attn_ms = timed(attn_run, args.steps, args.warmup)
-        build_ms = timed(build, args.steps, args.warmup)
-        dense_ms = timed(dense_run, args.steps, args.warmup)
-        compact_ms = timed(compact_step, args.steps, args.warmup)
-        gather_ms = timed(gather, args.steps, args.warmup)
-        tile_ms = timed(tile_step, args.steps, args.warmup)
-        tile_build_ms = timed(tile_build, args.steps, args.warmup)
-        build_bits_ms = timed(build_bits, args.steps, args.warmup)
-        build()  # the FP8 runs read this step's tables
-        fp8_ms = timed(fp8_attend, args.steps, args.warmup)
-        fp8_dense_ms = timed(fp8_dense, args.steps, args.warmup)
+        (step_ms, attn_ms, build_ms, dense_ms, compact_ms, gather_ms, tile_ms, tile_build_ms,
+         build_bits_ms, fp8_ms, fp8_dense_ms) = timed_round_robin(
+            [step_run, attn_run, build, dense_run, compact_step, gather, tile_step, tile_build,
+             build_bits, fp8_attend, fp8_dense], args.steps, args.warmup)
     clocks = clk.summary()
     assert ca.read_device_status(ws) == ca.CA_OK, "device status not OK"
 

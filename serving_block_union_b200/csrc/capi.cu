@@ -69,7 +69,7 @@ const char *ca_status_string(int status) {
     }
 }
 
-int ca_version(void) { return 100; }
+int ca_version(void) { return 200; }
 
 size_t ca_workspace_bytes(int B, int H_q, int H_kv, int C, int blk) {
     if (B <= 0 || H_q <= 0 || H_kv <= 0 || C <= 0 || blk <= 0 || H_q % H_kv != 0) return 0;
