@@ -264,7 +264,8 @@ def _config(wl, name=None, n_chunks=1):
            "l2": "256 MB L2 flush between timed steps; K/V cache larger than L2"}
     if n_chunks > 1:
         cfg["chunks_per_step"] = n_chunks
-        cfg["cuda_graph"] = "zero-copy step, attention and dense step replayed as CUDA graphs"
+        cfg["cuda_graph"] = ("every multi-chunk step (zero-copy, attention, dense, both "
+                             "ablations, FP8) replayed as a CUDA graph")
         cfg["cached_tokens"] = f"0..{wl.chunk_start[0]} (chunk k starts at {wl.C}*k)"
     return cfg
 
@@ -491,6 +492,8 @@ def run_ours(args, chunks):
         return g.replay
 
     step_run, attn_run, dense_run = graphed(step), graphed(attend), graphed(dense)
+    compact_run, tile_run = graphed(compact_step), graphed(tile_step)
+    fp8_run, fp8_dense_run = graphed(fp8_attend), graphed(fp8_dense)
     # Every path is timed in each step, round robin, so that all of them see
     # the same clocks and power state (a path timed alone in its own loop gets
     # whatever the loops before it left: the 1 kW power cap lowers the clocks
@@ -498,8 +501,8 @@ def run_ours(args, chunks):
     with ClockSampler(gpu_index) as clk:
         (step_ms, attn_ms, build_ms, dense_ms, compact_ms, gather_ms, tile_ms, tile_build_ms,
          build_bits_ms, fp8_ms, fp8_dense_ms) = timed_round_robin(
-            [step_run, attn_run, build, dense_run, compact_step, gather, tile_step, tile_build,
-             build_bits, fp8_attend, fp8_dense], args.steps, args.warmup)
+            [step_run, attn_run, build, dense_run, compact_run, gather, tile_run, tile_build,
+             build_bits, fp8_run, fp8_dense_run], args.steps, args.warmup)
     clocks = clk.summary()
     assert ca.read_device_status(ws) == ca.CA_OK, "device status not OK"
 
