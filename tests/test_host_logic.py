@@ -61,6 +61,30 @@ def test_pack_mask_bits_round_trip():
             assert sum(x << (32 * i) for i, x in enumerate(words)) == value
 
 
+def test_profiled_traffic_needs_matching_kernel_hash(tmp_path, monkeypatch):
+    """The roofline traffic field comes from a committed ncu summary only when
+    that summary was captured from the current kernel code; comment-only edits
+    of the kernel keep the hash."""
+    monkeypatch.setattr(bench, "PROFILES", str(tmp_path))
+    h = bench.kernel_source_hash()
+    (tmp_path / "chunk_attn_kernel_w.md").write_text(
+        f"text\n```\ndram_bytes_per_launch: 1234\nsource_sha256_16: {h}\n```\n")
+    assert bench.profiled_traffic("w") == 1234
+    (tmp_path / "chunk_attn_kernel_w.md").write_text(
+        "dram_bytes_per_launch: 1234\nsource_sha256_16: 0000000000000000\n")
+    assert bench.profiled_traffic("w") is None
+    assert bench.profiled_traffic("missing") is None
+    # comments and whitespace do not change the hash
+    src = tmp_path / "k.cu"
+    src.write_text("int a; // one\n/* two */ int  b;\n")
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", [str(src)])
+    h1 = bench.kernel_source_hash()
+    src.write_text("int a;   // changed comment\nint b;\n")
+    assert bench.kernel_source_hash() == h1
+    src.write_text("int a; int c;\n")
+    assert bench.kernel_source_hash() != h1
+
+
 def _poly_coeffs():
     src = open(os.path.join(ROOT, "serving_block_union_b200", "csrc", "sm100_ptx.cuh")).read()
     body = src[src.index("float exp2_poly(float x)"):]
