@@ -59,6 +59,8 @@ def _load():
             lib.oracle_attention_rows_e4m3.restype = I
             lib.oracle_e4m3_decode.argtypes = [I]
             lib.oracle_e4m3_decode.restype = ctypes.c_double
+            lib.oracle_merge_states.argtypes = [P, P, P, P, ctypes.c_int64, I, P, P]
+            lib.oracle_merge_states.restype = I
             lib.oracle_tile_span_tables.argtypes = [P, I, I, I, I, I, P, P]
             lib.oracle_tile_span_tables.restype = I
             lib.oracle_visible_pairs.argtypes = [P, P, P, I, I, I, I, I, I]
@@ -237,6 +239,27 @@ def attention_tile(Q, K, V, chunk_start: Sequence[int], blk: int, mask,
         raise ValueError(f"oracle_attention_tile_rows failed ({st})")
     if rows is None:
         return O.reshape(B, H_q, C, D), LSE.reshape(B, H_q, C)
+    return O, LSE
+
+
+def merge_states(O_a, LSE_a, O_b, LSE_b) -> Tuple[np.ndarray, np.ndarray]:
+    """Merge of two attention results over disjoint key sets (fp64): returns
+    ``O, LSE`` with ``LSE = ln(e^LSE_a + e^LSE_b)`` and ``O`` the
+    ``e^(LSE_x - LSE)``-weighted sum. Shapes ``[..., D]`` and ``[...]``."""
+    oa = np.ascontiguousarray(O_a, dtype=np.float64)
+    ob = np.ascontiguousarray(O_b, dtype=np.float64)
+    la = np.ascontiguousarray(LSE_a, dtype=np.float64)
+    lb = np.ascontiguousarray(LSE_b, dtype=np.float64)
+    if oa.shape != ob.shape or la.shape != lb.shape or oa.shape[:-1] != la.shape:
+        raise ValueError("shape mismatch")
+    D = oa.shape[-1]
+    rows = la.size
+    O = np.empty_like(oa)
+    LSE = np.empty_like(la)
+    st = _load().oracle_merge_states(_ptr(oa), _ptr(la), _ptr(ob), _ptr(lb), rows, D, _ptr(O),
+                                     _ptr(LSE))
+    if st != 0:
+        raise ValueError(f"oracle_merge_states failed ({st})")
     return O, LSE
 
 

@@ -374,6 +374,34 @@ int oracle_attention_tile_rows(const uint16_t *Q, const uint16_t *K, const uint1
 }
 
 /*
+ * Merge of two attention results over disjoint key sets of the same query
+ * rows (the identity the split-KV path rests on): with w_x = exp(LSE_x - L),
+ *     L = ln(exp(LSE_a) + exp(LSE_b)),   O = w_a O_a + w_b O_b,
+ * evaluated with the larger LSE subtracted first; two empty inputs (LSE =
+ * -inf) give O = 0, LSE = -inf. O_a, O_b, O fp64 [rows, D]; LSE fp64 [rows].
+ */
+int oracle_merge_states(const double *O_a, const double *LSE_a, const double *O_b,
+                        const double *LSE_b, int64_t rows, int D, double *O, double *LSE) {
+    if (!O_a || !LSE_a || !O_b || !LSE_b || !O || !LSE || rows < 0 || D <= 0)
+        return ORACLE_EINVAL;
+    for (int64_t r = 0; r < rows; ++r) {
+        const double la = LSE_a[r], lb = LSE_b[r];
+        const double m = la > lb ? la : lb;
+        if (m == -INFINITY) {
+            for (int d = 0; d < D; ++d) O[r * D + d] = 0.0;
+            LSE[r] = -INFINITY;
+            continue;
+        }
+        const double wa = exp(la - m), wb = exp(lb - m);
+        const double sum = wa + wb;
+        for (int d = 0; d < D; ++d)
+            O[r * D + d] = (wa * O_a[r * D + d] + wb * O_b[r * D + d]) / sum;
+        LSE[r] = m + log(sum);
+    }
+    return ORACLE_OK;
+}
+
+/*
  * Span tables for the per-tile path. The chunk's Q-blocks are taken in spans
  * of `span` consecutive Q-blocks (the last span may be short); for each
  * (b, h, span) the table lists, ascending, every KV block j that some

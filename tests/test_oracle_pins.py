@@ -356,6 +356,48 @@ def test_lse_merge_identity():
     np.testing.assert_allclose(Lm, L_, rtol=1e-12, atol=1e-12)
 
 
+def test_merge_states_pins():
+    """The oracle's state merge: disjoint halves merged equal attention over
+    the union; the special cases (one side empty, equal LSEs, both empty,
+    LSEs far beyond exp's range) have closed forms."""
+    B, H_q, H_kv, D, blk, C, L = 1, 2, 1, 16, 8, 16, 64
+    cs = (48,)
+    Q, K, V = _rand_qkv(22, B, H_q, H_kv, C, L, D)
+    nK = L // blk
+    full = np.array([[[0, 2, 3, 5, 6, 7] + [-1] * (nK - 6)]], np.int32)
+    a = np.array([[[2, 5, 7] + [-1] * (nK - 3)]], np.int32)
+    bb = np.array([[[0, 3, 6] + [-1] * (nK - 3)]], np.int32)
+    n6, n3 = np.array([[6]], np.int32), np.array([[3]], np.int32)
+    O, L_ = oracle.attention(Q, K, V, cs, blk, full, n6)
+    O1, L1 = oracle.attention(Q, K, V, cs, blk, a, n3)
+    O2, L2 = oracle.attention(Q, K, V, cs, blk, bb, n3)
+    Om, Lm = oracle.merge_states(O1, L1, O2, L2)
+    np.testing.assert_allclose(Om, O, rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(Lm, L_, rtol=1e-12, atol=1e-12)
+    Os, Ls = oracle.merge_states(O2, L2, O1, L1)  # symmetric
+    np.testing.assert_allclose(Os, Om, rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(Ls, Lm, rtol=1e-14, atol=1e-14)
+
+    rng = np.random.default_rng(5)
+    Oa, Ob = rng.standard_normal((2, 6, 4))
+    la = np.array([0.0, -3.0, 2.5, 1000.0, -1000.0, -np.inf])
+    inf = np.full(6, -np.inf)
+    O, Lz = oracle.merge_states(Oa, la, Ob, inf)       # other side empty
+    np.testing.assert_array_equal(O[:5], Oa[:5])
+    np.testing.assert_array_equal(Lz[:5], la[:5])
+    assert np.all(O[5] == 0.0) and Lz[5] == -np.inf   # both empty
+    O, Le = oracle.merge_states(Oa[:5], la[:5], Ob[:5], la[:5].copy())
+    np.testing.assert_allclose(O, (Oa[:5] + Ob[:5]) / 2, rtol=1e-15, atol=1e-15)
+    np.testing.assert_allclose(Le, la[:5] + math.log(2.0), rtol=1e-15, atol=1e-12)
+    # weights e/(1+e) and 1/(1+e) at an LSE gap of 1, far from exp's range
+    O, Lg = oracle.merge_states(Oa[3:5], la[3:5] + 1.0, Ob[3:5], la[3:5])
+    w = math.e / (1.0 + math.e)
+    np.testing.assert_allclose(O, w * Oa[3:5] + (1 - w) * Ob[3:5], rtol=1e-14, atol=1e-14)
+    np.testing.assert_allclose(Lg, la[3:5] + 1.0 + math.log1p(math.exp(-1.0)), rtol=1e-15)
+    with pytest.raises(ValueError):
+        oracle.merge_states(Oa, la, Ob[:5], la[:5])
+
+
 def test_nan_poison_outside_visible_keys_is_never_read():
     B, H_q, H_kv, D, blk, C, L = 2, 4, 1, 8, 4, 8, 48
     cs = (16, 32)
