@@ -81,6 +81,30 @@ def profiled_traffic(workload: str):
         return None
 
 
+def _merge_line(O, ms, O_big, ms_big, peaks, peak_kind):
+    """The two-part state merge: algorithmic bytes per row = two bf16 O rows
+    and two fp32 LSEs read, one O row and one LSE written (6 D + 12)."""
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+
+    def one(o, t_ms):
+        D = o.shape[-1]
+        rows = o.numel() // D
+        byts = rows * (6 * D + 12)
+        gbs = byts / (t_ms * 1e-3) / 1e9
+        return {"rows": rows, "D": D, "us": t_ms * 1e3, "bytes": byts, "gbs": gbs,
+                "frac_of_hbm": gbs / hbm}
+
+    line = one(O, ms)
+    line["note"] = ("this chunk's result shape; inputs read from HBM (L2 flushed), the "
+                    "output may still sit in L2 when the timer stops")
+    big = one(O_big, ms_big)
+    big["note"] = "traffic well above L2: the HBM roofline of the merge kernel"
+    line["large"] = big
+    line["parts"] = 2
+    line["peak_source"] = f"{peak_kind} HBM copy bandwidth"
+    return line
+
+
 def _peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -491,6 +515,27 @@ def run_ours(args, chunks):
         graphs.append(g)
         return g.replay
 
+    # Merge of two attention states (split-KV across calls or GPUs): the
+    # chunk's own result shape, and a large one (1M rows) whose traffic is
+    # well above L2, for the HBM roofline of the merge kernel.
+    attend()
+    torch.cuda.synchronize(dev)
+    mg = torch.Generator(device=dev).manual_seed(1234)
+    m_parts = [(Os[0], LSEs[0]),
+               (torch.randn(Os[0].shape, generator=mg, device=dev).to(torch.bfloat16),
+                torch.randn(LSEs[0].shape, generator=mg, device=dev) * 4)]
+    m_out = (torch.empty_like(Os[0]), torch.empty_like(LSEs[0]))
+    big_rows, mD = 1 << 20, wl0.D
+    big_parts = [(torch.randn(big_rows, mD, generator=mg, device=dev).to(torch.bfloat16),
+                  torch.randn(big_rows, generator=mg, device=dev) * 4) for _ in range(2)]
+    big_out = (torch.empty_like(big_parts[0][0]), torch.empty_like(big_parts[0][1]))
+
+    def merge():
+        ca.merge_attention_states(m_parts, O=m_out[0], LSE=m_out[1], stream=stream)
+
+    def merge_big():
+        ca.merge_attention_states(big_parts, O=big_out[0], LSE=big_out[1], stream=stream)
+
     step_run, attn_run, dense_run = graphed(step), graphed(attend), graphed(dense)
     compact_run, tile_run = graphed(compact_step), graphed(tile_step)
     fp8_run, fp8_dense_run = graphed(fp8_attend), graphed(fp8_dense)
@@ -500,9 +545,9 @@ def run_ours(args, chunks):
     # as the run heats up). build_bits rewrites the tables the FP8 runs read.
     with ClockSampler(gpu_index) as clk:
         (step_ms, attn_ms, build_ms, dense_ms, compact_ms, gather_ms, tile_ms, tile_build_ms,
-         build_bits_ms, fp8_ms, fp8_dense_ms) = timed_round_robin(
+         build_bits_ms, fp8_ms, fp8_dense_ms, merge_ms, merge_big_ms) = timed_round_robin(
             [step_run, attn_run, build, dense_run, compact_run, gather, tile_run, tile_build,
-             build_bits, fp8_run, fp8_dense_run], args.steps, args.warmup)
+             build_bits, fp8_run, fp8_dense_run, merge, merge_big], args.steps, args.warmup)
     clocks = clk.summary()
     assert ca.read_device_status(ws) == ca.CA_OK, "device status not OK"
 
@@ -605,6 +650,8 @@ def run_ours(args, chunks):
     total_build_bits = agg(build_bits_ms)
     total_fp8 = agg(fp8_ms)
     total_fp8_dense = agg(fp8_dense_ms)
+    total_merge = agg(merge_ms)
+    total_merge_big = agg(merge_big_ms)
     K_ = args.steps
     value = world * K_ * flops / (total_step * 1e-3) / 1e12
     attn_tflops = flops / (total_attn / K_ * 1e-3) / 1e12
@@ -645,6 +692,8 @@ def run_ours(args, chunks):
             "speedup_vs_dense_fp8": total_fp8_dense / total_fp8,
             "speedup_vs_bf16_attention": total_attn / total_fp8,
             "note": "Q, K, V per-tensor E4M3 (amax / 448 descale), same tables"},
+        "merge_states": _merge_line(m_out[0], total_merge / K_, big_out[0], total_merge_big / K_,
+                                    peaks, peak_kind),
         "effective_tflop_per_step": flops / 1e12,
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": attn_tflops / peak,

@@ -308,6 +308,42 @@ int ca_chunk_attention_noalloc(const void *Q, const void *K, const void *V, cons
                                int H_kv, int C, int L_max, int D, int blk, float scale, void *O,
                                float *LSE, unsigned int *device_status, void *stream);
 
+/*
+ * Merge of attention results over disjoint key sets (CompactAttention pages,
+ * "Implementation": split-KV execution cuts one query row's attention over
+ * several segments of its KV blocks and merges them by their log-sum-exp).
+ * Each part i holds, for the same query rows, O_i normalised over its own
+ * keys and LSE_i = ln sum exp(score) over them (natural log, the convention of
+ * ca_chunk_attention's LSE output). The merged result is attention over the
+ * union of the key sets:
+ *     LSE[r]   = ln sum_i exp(LSE_i[r])
+ *     O[r, :]  = sum_i exp(LSE_i[r] - LSE[r]) * O_i[r, :]
+ * computed in fp32 with the largest LSE_i[r] subtracted first. A part with
+ * LSE_i[r] = -inf (no visible key) has weight 0; if every part has -inf the
+ * row gets O = 0, LSE = -inf. LSE_i must be finite or -inf.
+ *
+ * O_a, O_b, O  bf16 [rows, D] row-major (any leading shape flattened to rows,
+ *              e.g. [B, H_q, C] of ca_chunk_attention), 16-byte aligned;
+ * LSE_a, LSE_b fp32 [rows], 4-byte aligned; LSE fp32 [rows] or NULL (not
+ *              written). O may be the same buffer as O_a or O_b (in place) and
+ *              LSE the same as LSE_a or LSE_b; partial overlaps are not allowed.
+ * D: a multiple of 8, at most 2048. rows == 0 is a no-op. All pointers are
+ * device memory owned by the caller; the call is asynchronous on `stream`.
+ * Errors: CA_ERR_INVALID_ARG (NULL input / negative rows / D <= 0),
+ * CA_ERR_SHAPE (D not a multiple of 8), CA_ERR_UNSUPPORTED (D > 2048),
+ * CA_ERR_ALIGN, CA_ERR_CUDA (launch failure).
+ */
+int ca_merge_attention_states(const void *O_a, const float *LSE_a, const void *O_b,
+                              const float *LSE_b, long long rows, int D, void *O, float *LSE,
+                              void *stream);
+
+/* The same merge over n parts (2 <= n <= 8, else CA_ERR_UNSUPPORTED; n == 1
+ * is CA_ERR_INVALID_ARG). O_parts / LSE_parts are HOST arrays of n device
+ * pointers (read during the call only), each part laid out as O_a / LSE_a
+ * above. One pass over the data: no intermediate rounding to bf16. */
+int ca_merge_attention_states_n(const void *const *O_parts, const float *const *LSE_parts, int n,
+                                long long rows, int D, void *O, float *LSE, void *stream);
+
 /* Self-test of the kernels' bounded waits: one kernel waits on a barrier that
  * nothing ever completes; after limit_cycles SM clock cycles (at most about
  * 2 s) the wait gives up, sets the timeout bit of the workspace status word

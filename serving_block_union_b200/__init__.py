@@ -38,6 +38,15 @@ __all__ = [
     "chunk_attention_noalloc",
     "compact_kv_blocks",
     "compacted_chunk_attention",
+    "build_block_tables_bits",
+    "build_kv_pages",
+    "selftest_bounded_wait",
+    "tile_span",
+    "build_tile_tables",
+    "tile_chunk_attention",
+    "paged_chunk_attention",
+    "chunk_attention_fp8",
+    "merge_attention_states",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -76,6 +85,8 @@ EXPORTED_SYMBOLS = (
     "ca_paged_chunk_attention",
     "ca_build_tile_tables",
     "ca_tile_chunk_attention",
+    "ca_merge_attention_states",
+    "ca_merge_attention_states_n",
 )
 
 
@@ -141,6 +152,10 @@ def load_library():
         lib.ca_tile_chunk_attention.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, P, P, P,
                                                 S, P]
         lib.ca_tile_chunk_attention.restype = I
+        lib.ca_merge_attention_states.argtypes = [P, P, P, P, ctypes.c_longlong, I, P, P, P]
+        lib.ca_merge_attention_states.restype = I
+        lib.ca_merge_attention_states_n.argtypes = [P, P, I, ctypes.c_longlong, I, P, P, P]
+        lib.ca_merge_attention_states_n.restype = I
         _lib = lib
         return lib
 
@@ -638,4 +653,49 @@ def chunk_attention_fp8(Q8: torch.Tensor, K8: torch.Tensor, V8: torch.Tensor,
         C, L_max, D, int(blk), float(scale), _ptr(O), _ptr(LSE), _ptr(workspace),
         workspace.numel(), _stream_handle(stream, dev))
     _check("ca_chunk_attention_fp8", st)
+    return O, LSE
+
+
+# ----------------------------------------------------------------- merge
+
+def merge_attention_states(parts: Sequence[Tuple[torch.Tensor, torch.Tensor]],
+                           O: Optional[torch.Tensor] = None, LSE: Optional[torch.Tensor] = None,
+                           want_lse: bool = True, stream: Optional[torch.cuda.Stream] = None
+                           ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Merges attention results over disjoint key sets of the same query rows:
+    ``parts`` = [(O_i bf16 [..., D], LSE_i fp32 [...]), ...] (2 to 8 parts, as
+    ``chunk_attention`` returns them) -> attention over the union of the key
+    sets, ``LSE = ln sum exp(LSE_i)``, ``O = sum exp(LSE_i - LSE) O_i``. ``O`` /
+    ``LSE`` may be given (also one of the parts' own tensors, for in place);
+    with ``want_lse=False`` and no ``LSE`` the merged LSE is not written."""
+    parts = list(parts)
+    if len(parts) < 2:
+        raise ValueError("merge_attention_states needs at least two parts")
+    O0, L0 = parts[0]
+    shape = tuple(O0.shape)
+    for i, (Oi, Li) in enumerate(parts):
+        _need(Oi, f"O_{i}", torch.bfloat16, len(shape))
+        _need(Li, f"LSE_{i}", torch.float32, len(shape) - 1)
+        if tuple(Oi.shape) != shape or tuple(Li.shape) != shape[:-1]:
+            raise ValueError(f"part {i}: shapes {tuple(Oi.shape)} / {tuple(Li.shape)} "
+                             f"do not match {shape} / {shape[:-1]}")
+    D = shape[-1]
+    rows = O0.numel() // D if D else 0
+    if O is None:
+        O = torch.empty_like(O0)
+    _need(O, "O", torch.bfloat16, len(shape))
+    if tuple(O.shape) != shape:
+        raise ValueError(f"O must have shape {shape}")
+    if LSE is None and want_lse:
+        LSE = torch.empty_like(L0)
+    if LSE is not None:
+        _need(LSE, "LSE", torch.float32, len(shape) - 1)
+        if tuple(LSE.shape) != shape[:-1]:
+            raise ValueError(f"LSE must have shape {shape[:-1]}")
+    n = len(parts)
+    o_arr = (ctypes.c_void_p * n)(*[Oi.data_ptr() for Oi, _ in parts])
+    l_arr = (ctypes.c_void_p * n)(*[Li.data_ptr() for _, Li in parts])
+    st = load_library().ca_merge_attention_states_n(o_arr, l_arr, n, rows, D, _ptr(O), _ptr(LSE),
+                                                    _stream_handle(stream, O0.device))
+    _check("ca_merge_attention_states_n", st)
     return O, LSE

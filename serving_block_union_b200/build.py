@@ -18,7 +18,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libcompactattn.so")
 SOURCES = ["capi.cu", "build_tables.cu", "chunk_attention.cu", "compact_kv.cu", "noalloc.cu",
-           "selftest.cu", "tile_tables.cu"]
+           "merge_states.cu", "selftest.cu", "tile_tables.cu"]
 HEADERS = ["ca_internal.h", "sm100_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -147,4 +147,10 @@ int launch_compact_kv(const void *K, const void *V, const int32_t *tables, const
                       int B, int H_kv, int L_max, int D, int blk, void *Kc, void *Vc,
                       cudaStream_t stream);
 
+// Merge of n attention results over disjoint key sets (2 <= n <= kMaxMergeParts):
+// LSE = ln sum_i exp(LSE_i), O = sum_i exp(LSE_i - LSE) O_i; bf16 O, fp32 LSE.
+constexpr int kMaxMergeParts = 8;
+int launch_merge_states(const void *const *O_parts, const float *const *LSE_parts, int n,
+                        long long rows, int D, void *O, float *LSE, cudaStream_t stream);
+
 }  // namespace ca

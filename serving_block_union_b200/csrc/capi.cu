@@ -226,6 +226,29 @@ int ca_compacted_chunk_attention(const void *Q, const void *Kc, const void *Vc,
     return ca::launch_chunk_attention(a, ca::kModeCompact, static_cast<cudaStream_t>(stream));
 }
 
+int ca_merge_attention_states_n(const void *const *O_parts, const float *const *LSE_parts, int n,
+                                long long rows, int D, void *O, float *LSE, void *stream) {
+    if (!O_parts || !LSE_parts || !O || n < 2 || rows < 0 || D <= 0) return CA_ERR_INVALID_ARG;
+    if (n > ca::kMaxMergeParts) return CA_ERR_UNSUPPORTED;
+    if (D % 8 != 0) return CA_ERR_SHAPE;
+    if (D > 2048) return CA_ERR_UNSUPPORTED;
+    for (int i = 0; i < n; ++i) {
+        if (!O_parts[i] || !LSE_parts[i]) return CA_ERR_INVALID_ARG;
+        if (!aligned(O_parts[i], 16) || !aligned(LSE_parts[i], 4)) return CA_ERR_ALIGN;
+    }
+    if (!aligned(O, 16) || (LSE && !aligned(LSE, 4))) return CA_ERR_ALIGN;
+    return ca::launch_merge_states(O_parts, LSE_parts, n, rows, D, O, LSE,
+                                   static_cast<cudaStream_t>(stream));
+}
+
+int ca_merge_attention_states(const void *O_a, const float *LSE_a, const void *O_b,
+                              const float *LSE_b, long long rows, int D, void *O, float *LSE,
+                              void *stream) {
+    const void *o[2] = {O_a, O_b};
+    const float *l[2] = {LSE_a, LSE_b};
+    return ca_merge_attention_states_n(o, l, 2, rows, D, O, LSE, stream);
+}
+
 int ca_tile_span(int blk) {
     return (blk == 64 || blk == 128) ? ca::kTileItemRows / blk : 0;
 }

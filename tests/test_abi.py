@@ -166,6 +166,30 @@ def test_paged_path_host_checks(lib):
              A16, A16, 256, None) == ca.CA_ERR_SHAPE
 
 
+def test_merge_states_host_checks(lib):
+    f = lib.ca_merge_attention_states
+    assert f(None, A16, A16, A16, 10, 128, A16, A16, None) == ca.CA_ERR_INVALID_ARG
+    assert f(A16, None, A16, A16, 10, 128, A16, A16, None) == ca.CA_ERR_INVALID_ARG
+    assert f(A16, A16, A16, A16, 10, 128, None, A16, None) == ca.CA_ERR_INVALID_ARG
+    assert f(A16, A16, A16, A16, -1, 128, A16, A16, None) == ca.CA_ERR_INVALID_ARG
+    assert f(A16, A16, A16, A16, 10, 0, A16, A16, None) == ca.CA_ERR_INVALID_ARG
+    assert f(A16, A16, A16, A16, 10, 100, A16, A16, None) == ca.CA_ERR_SHAPE
+    assert f(A16, A16, A16, A16, 10, 4096, A16, A16, None) == ca.CA_ERR_UNSUPPORTED
+    assert f(A_MIS, A16, A16, A16, 10, 128, A16, A16, None) == ca.CA_ERR_ALIGN
+    assert f(A16, A16, A16, A16, 10, 128, A_MIS, A16, None) == ca.CA_ERR_ALIGN
+    assert f(A16, ctypes.c_void_p((1 << 20) + 2), A16, A16, 10, 128, A16, A16,
+             None) == ca.CA_ERR_ALIGN
+    assert f(A16, A16, A16, A16, 0, 128, A16, None, None) == ca.CA_OK   # empty: no launch
+    g = lib.ca_merge_attention_states_n
+    arr = (ctypes.c_void_p * 9)(*([A16.value] * 9))
+    assert g(arr, arr, 1, 10, 128, A16, A16, None) == ca.CA_ERR_INVALID_ARG
+    assert g(arr, arr, 9, 10, 128, A16, A16, None) == ca.CA_ERR_UNSUPPORTED
+    assert g(None, arr, 2, 10, 128, A16, A16, None) == ca.CA_ERR_INVALID_ARG
+    holey = (ctypes.c_void_p * 3)(A16.value, None, A16.value)
+    assert g(holey, arr, 3, 10, 128, A16, A16, None) == ca.CA_ERR_INVALID_ARG
+    assert g(arr, arr, 8, 0, 64, A16, A16, None) == ca.CA_OK
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     import importlib
     monkeypatch.setattr(ca, "_lib", None)
