@@ -105,6 +105,11 @@ def _merge_line(O, ms, O_big, ms_big, peaks, peak_kind):
     return line
 
 
+def peaks_hbm():
+    p, kind = _peaks()
+    return float(p.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])), kind
+
+
 def _peaks():
     try:
         with open(PEAKS_FILE) as f:
@@ -132,6 +137,41 @@ def visible_pairs(tables: np.ndarray, counts: np.ndarray, chunk_start, C: int, b
             vis = np.clip(p[:, None] - starts[None, :] + 1, 0, blk)
             total += int(vis.sum()) * G
     return total
+
+
+def executed_pairs(tables: np.ndarray, counts: np.ndarray, chunk_start, C: int, blk: int,
+                   G: int, dense_nkv=None) -> int:
+    """(row, key) pairs the tensor core multiplies, whole tiles counted: the
+    kernel's work item is two 128-row tiles of packed (chunk row, head) pairs
+    of one group (128 / G chunk rows per tile); it walks the table entries
+    whose block starts at or before the item's last position, every tile of
+    it against every key of each such block (the causal diagonal included in
+    full)."""
+    B, H_kv = counts.shape
+    R = 128 // G
+    total = 0
+    for b in range(B):
+        for g in range(H_kv):
+            if dense_nkv is not None:
+                starts = np.arange(dense_nkv[b], dtype=np.int64) * blk
+            else:
+                starts = np.sort(tables[b, g, : counts[b, g]].astype(np.int64)) * blk
+            for r0 in range(0, C, 2 * R):
+                last = chunk_start[b] + min(r0 + 2 * R, C) - 1
+                n_eff = int(np.searchsorted(starts, last, side="right"))
+                total += n_eff * 2 * 128 * blk
+    return total
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def tile_visible_pairs(mask: np.ndarray, chunk_start, C: int, blk: int) -> int:
@@ -273,7 +313,7 @@ def run_reference(args, wl, name=None):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": _config(wl, name),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu_model": cpu_model(), "nproc": os.cpu_count()},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -473,7 +513,7 @@ def run_ours(args, chunks):
     # work count of one step (from the step's own tables)
     build()
     torch.cuda.synchronize(dev)
-    flops = dense_flops = tile_flops = 0.0
+    flops = dense_flops = tile_flops = exec_flops = dense_exec_flops = 0.0
     union_num = union_den = 0
     table_bytes = 0
     for k, w in enumerate(chunks):
@@ -482,6 +522,10 @@ def run_ours(args, chunks):
         flops += 4.0 * w.D * visible_pairs(T_np, c_np, w.chunk_start, w.C, w.blk, w.group)
         dense_flops += 4.0 * w.D * visible_pairs(T_np, c_np, w.chunk_start, w.C, w.blk, w.group,
                                                  dense_nkv=nkv)
+        exec_flops += 4.0 * w.D * executed_pairs(T_np, c_np, w.chunk_start, w.C, w.blk,
+                                                 w.group)
+        dense_exec_flops += 4.0 * w.D * executed_pairs(T_np, c_np, w.chunk_start, w.C, w.blk,
+                                                       w.group, dense_nkv=nkv)
         union_num += int(c_np.sum())
         union_den += sum(nkv) * w.H_kv
         table_bytes += masks_np[k].nbytes + 4 * T_np.size + 4 * c_np.size
@@ -533,6 +577,24 @@ def run_ours(args, chunks):
     def merge():
         ca.merge_attention_states(m_parts, O=m_out[0], LSE=m_out[1], stream=stream)
 
+    # the table build at a size where bandwidth is measurable: 64 sequences of
+    # this shape at 128K (16 Q-blocks, 1040 KV blocks), 10% Bernoulli mask
+    st_B, st_nQ, st_nK = 64, 16, 1040
+    st_np = (np.random.default_rng(77).random((st_B, wl0.H_q, st_nQ, st_nK)) < 0.1).astype(
+        np.uint8)
+    st_mask = torch.from_numpy(st_np).to(dev)
+    st_bits = torch.from_numpy(workloads.pack_mask_bits(st_np).view(np.int32)).to(dev)
+    del st_np
+    st_T = torch.empty((st_B, wl0.H_kv, st_nK), dtype=torch.int32, device=dev)
+    st_c = torch.empty((st_B, wl0.H_kv), dtype=torch.int32, device=dev)
+
+    def build_stress():
+        ca.build_block_tables(st_mask, wl0.group, tables=st_T, counts=st_c, stream=stream)
+
+    def build_stress_bits():
+        ca.build_block_tables_bits(st_bits, st_nK, wl0.group, tables=st_T, counts=st_c,
+                                   stream=stream)
+
     def merge_big():
         ca.merge_attention_states(big_parts, O=big_out[0], LSE=big_out[1], stream=stream)
 
@@ -545,9 +607,11 @@ def run_ours(args, chunks):
     # as the run heats up). build_bits rewrites the tables the FP8 runs read.
     with ClockSampler(gpu_index) as clk:
         (step_ms, attn_ms, build_ms, dense_ms, compact_ms, gather_ms, tile_ms, tile_build_ms,
-         build_bits_ms, fp8_ms, fp8_dense_ms, merge_ms, merge_big_ms) = timed_round_robin(
+         build_bits_ms, fp8_ms, fp8_dense_ms, merge_ms, merge_big_ms, stress_ms,
+         stress_bits_ms) = timed_round_robin(
             [step_run, attn_run, build, dense_run, compact_run, gather, tile_run, tile_build,
-             build_bits, fp8_run, fp8_dense_run, merge, merge_big], args.steps, args.warmup)
+             build_bits, fp8_run, fp8_dense_run, merge, merge_big, build_stress,
+             build_stress_bits], args.steps, args.warmup)
     clocks = clk.summary()
     assert ca.read_device_status(ws) == ca.CA_OK, "device status not OK"
 
@@ -652,6 +716,20 @@ def run_ours(args, chunks):
     total_fp8_dense = agg(fp8_dense_ms)
     total_merge = agg(merge_ms)
     total_merge_big = agg(merge_big_ms)
+    total_stress = agg(stress_ms)
+    total_stress_bits = agg(stress_bits_ms)
+    hbm_peak = float(peaks_hbm()[0])
+    st_out = st_T.numel() * 4 + st_c.numel() * 4
+    st_us, st_bits_us = total_stress / args.steps * 1e3, total_stress_bits / args.steps * 1e3
+    build_stress_line = {
+        "B": st_B, "H_q": wl0.H_q, "nQ": st_nQ, "nKVmax": st_nK, "mask_density": 0.1,
+        "mask_bytes": st_mask.numel(), "out_bytes": st_out,
+        "us": st_us, "gbs": (st_mask.numel() + st_out) / (st_us * 1e-6) / 1e9,
+        "frac_of_hbm": (st_mask.numel() + st_out) / (st_us * 1e-6) / 1e9 / hbm_peak,
+        "bits_mask_bytes": st_bits.numel() * 4, "bits_us": st_bits_us,
+        "bits_gbs": (st_bits.numel() * 4 + st_out) / (st_bits_us * 1e-6) / 1e9,
+        "note": "table build where its bytes are measurable (the per-chunk build is "
+                "latency bound)"}
     K_ = args.steps
     value = world * K_ * flops / (total_step * 1e-3) / 1e12
     attn_tflops = flops / (total_attn / K_ * 1e-3) / 1e12
@@ -668,6 +746,7 @@ def run_ours(args, chunks):
         "build_us": total_build / K_ * 1e3,
         "build_gbs": table_bytes / (total_build / K_ * 1e-3) / 1e9,
         "build_bits_us": total_build_bits / K_ * 1e3,
+        "build_stress": build_stress_line,
         "dense_ms": total_dense / K_,
         "dense_tflops": dense_flops / (total_dense / K_ * 1e-3) / 1e12,
         "speedup_vs_dense": total_dense / total_step,
@@ -695,6 +774,14 @@ def run_ours(args, chunks):
         "merge_states": _merge_line(m_out[0], total_merge / K_, big_out[0], total_merge_big / K_,
                                     peaks, peak_kind),
         "effective_tflop_per_step": flops / 1e12,
+        "executed": {
+            "tflop_per_step": exec_flops / 1e12,
+            "attn_tflops": exec_flops / (total_attn / K_ * 1e-3) / 1e12,
+            "frac_of_peak": exec_flops / (total_attn / K_ * 1e-3) / 1e12 / peak,
+            "dense_tflop_per_step": dense_exec_flops / 1e12,
+            "dense_tflops": dense_exec_flops / (total_dense / K_ * 1e-3) / 1e12,
+            "note": "whole 128-row x block tiles the tensor core multiplies (causal "
+                    "diagonal counted in full), beside the effective (visible-pair) flops"},
         "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
                      "unit": "TFLOP/s", "frac": attn_tflops / peak,
                      "traffic": profiled_traffic(name) if n == 1 else None,
@@ -715,7 +802,8 @@ def run_ours(args, chunks):
                                                    target_s=args.cpu_seconds)
         line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                                 "sample": f"{nrows} seeded query rows of {last.B * last.H_q * last.C}"
-                                          f" of chunk {last.name} ({dt:.1f} s, fp64)"}
+                                          f" of chunk {last.name} ({dt:.1f} s, fp64)",
+                                "cpu_model": cpu_model(), "nproc": os.cpu_count()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -6,13 +6,16 @@
 // per-(batch, KV-group) table T_{b,g}; the CSR form is the kv_indptr /
 // kv_indices metadata handed to the paged kernel.
 //
-// One CTA per (b, g). Thread (rg, c) owns 16 consecutive KV blocks (chunk c)
+// Two forms. With few (b, g), each is spread over a cluster of CTAs (the
+// cluster kernel below). Otherwise one CTA per (b, g): thread (rg, c) owns 16
+// consecutive KV blocks (chunk c)
 // and ORs 16-byte vectors of the mask rows rg, rg + RG, ... of the group's
 // G * nQ rows (coalesced: consecutive threads read consecutive 16-byte words
 // of a row). Row groups are OR-combined through shared memory, every chunk
 // turns its 16 bytes into a 16-bit set, and a block-wide exclusive prefix sum
 // of the popcounts (warp shuffles + one shared-memory pass) gives each chunk
 // its write offset, so the table comes out ascending without a sort.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -23,6 +26,12 @@ namespace ca {
 namespace {
 
 constexpr int kMaxThreads = 1024;
+
+// The cluster form of the union (below) is the default; 0 keeps the one-CTA-
+// per-(b, g) form for every shape.
+#ifndef CA_BUILD_CLUSTER
+#define CA_BUILD_CLUSTER 1
+#endif
 
 __device__ __forceinline__ uint32_t nonzero_nibble(uint32_t w) {
     // 4 bits: bit k = (byte k of w != 0)
@@ -198,6 +207,144 @@ __global__ void __launch_bounds__(kMaxThreads)
     if (tid == 0) counts[bg] = n;
 }
 
+// Cluster form of the same union: a (b, g) row set is spread over a cluster of
+// kClusterCtas CTAs, CTA q taking units [q * upc, (q + 1) * upc) of the KV
+// range (a unit is 16 blocks of a byte mask, one 16-byte load per row, or 32
+// blocks of a bit mask, one 32-bit word per row). Each CTA ORs its units over
+// the group's G * nQ rows (one load per (row, unit) pair, consecutive threads
+// on consecutive units of a row, folded into shared memory by atomicOr), scans
+// its popcounts, and publishes its entry total in shared memory; after a
+// cluster barrier every CTA reads the totals of the others through
+// distributed shared memory, which gives its write offset and the table
+// length. A second cluster barrier keeps each CTA's shared memory alive until
+// the others have read it. So one (b, g) is read by kClusterCtas SMs at once
+// instead of one, and the table still comes out ascending without a sort.
+constexpr int kClusterCtas = 8;
+constexpr int kClusterThreads = 256;
+constexpr int kMaxUnitsPerCta = 1024;
+
+template <bool BITS>
+__global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterThreads)
+    union_tables_cluster_kernel(const void *__restrict__ mask, int H_q, int nQ, int nKVmax, int G,
+                                int upc, int32_t *__restrict__ tables,
+                                int32_t *__restrict__ counts) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    __shared__ uint32_t s_bits[kMaxUnitsPerCta];
+    __shared__ int s_off[kMaxUnitsPerCta];
+    __shared__ int warp_sums[32];
+    __shared__ int s_total, s_base, s_n;
+
+    constexpr int UB = BITS ? 32 : 16;  // KV blocks per unit
+    const int q = static_cast<int>(cluster.block_rank());
+    const int bg = blockIdx.y;
+    const int H_kv = H_q / G;
+    const int b = bg / H_kv, g = bg % H_kv;
+    const int tid = threadIdx.x;
+    const int n_units = (nKVmax + UB - 1) / UB;
+    const int u0 = q * upc;
+    const int nu = max(0, min(upc, n_units - u0));
+    const int n_rows = G * nQ;
+    const size_t row0 = ((size_t)b * H_q + (size_t)g * G) * nQ;
+    int32_t *T = tables + (size_t)bg * nKVmax;
+
+    for (int u = tid; u < nu; u += kClusterThreads) s_bits[u] = 0;
+    __syncthreads();
+    // pass 1: the union of this CTA's units, four (row, unit) loads in flight
+    // per thread before their results are folded in
+    const int pairs = n_rows * nu;
+    for (int p0 = tid; p0 < pairs; p0 += 4 * kClusterThreads) {
+        uint32_t bits[4];
+        int unit[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int p = p0 + k * kClusterThreads;
+            bits[k] = 0;
+            unit[k] = 0;
+            if (p < pairs) {
+                const int row = p / nu;
+                const int u = p - row * nu;
+                unit[k] = u;
+                if constexpr (BITS) {
+                    const int nW = n_units;
+                    bits[k] = __ldg(static_cast<const uint32_t *>(mask) + (row0 + row) * nW + u0 + u);
+                } else {
+                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
+                        static_cast<const uint8_t *>(mask) + (row0 + row) * (size_t)nKVmax +
+                        (size_t)(u0 + u) * 16));
+                    bits[k] = nonzero_bytes16(v);
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (bits[k]) atomicOr(&s_bits[unit[k]], bits[k]);
+    }
+    __syncthreads();
+    if constexpr (BITS) {
+        // bits at or past nKVmax name no block
+        if (tid == 0 && nu > 0) {
+            const int valid = nKVmax - (u0 + nu - 1) * 32;
+            if (valid < 32) s_bits[nu - 1] &= (1u << valid) - 1u;
+        }
+        __syncthreads();
+    }
+    // pass 2: CTA-local exclusive scan of the units' popcounts
+    int run = 0;
+    for (int r0 = 0; r0 < nu; r0 += kClusterThreads) {
+        const int u = r0 + tid;
+        const int c = u < nu ? __popc(s_bits[u]) : 0;
+        int tot = 0;
+        const int off = block_exclusive_scan(c, tid, kClusterThreads, warp_sums, &tot);
+        if (u < nu) s_off[u] = run + off;
+        run += tot;
+        __syncthreads();  // warp_sums is reused by the next round
+    }
+    if (tid == 0) s_total = run;
+    cluster.sync();
+    // this CTA's offset (totals of the lower ranks) and the table length
+    if (tid < 32) {
+        const int t = tid < kClusterCtas ? *cluster.map_shared_rank(&s_total, tid) : 0;
+        int below = tid < q ? t : 0;
+        int all = t;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            below += __shfl_xor_sync(0xffffffffu, below, o);
+            all += __shfl_xor_sync(0xffffffffu, all, o);
+        }
+        if (tid == 0) {
+            s_base = below;
+            s_n = all;
+        }
+    }
+    __syncthreads();
+    const int base = s_base, n = s_n;
+    for (int u = tid; u < nu; u += kClusterThreads) {
+        uint32_t m = s_bits[u];
+        int w = base + s_off[u];
+        const int j0 = (u0 + u) * UB;
+        while (m) {
+            const int k = __ffs(m) - 1;
+            T[w++] = j0 + k;
+            m &= m - 1;
+        }
+    }
+    for (int t = n + q * kClusterThreads + tid; t < nKVmax; t += kClusterCtas * kClusterThreads)
+        T[t] = -1;
+    if (q == 0 && tid == 0) counts[bg] = n;
+    cluster.sync();  // the other CTAs have read s_total before anyone exits
+}
+
+// Units per CTA of the cluster form, or 0 where it does not apply. It pays
+// only while one CTA per (b, g) leaves most SMs idle (a single sequence or a
+// few): measured at 128K (G = 4, 16 Q-blocks), 8 (b, g) build in 10.8 us
+// against 14.7 us with one CTA each, but 512 (b, g) take 36.6 us against 20.6.
+int cluster_upc(int n_units, int n_bg) {
+    if (n_bg <= 0 || n_bg > 65535 || n_bg > current_sm_count() / 4) return 0;
+    const int upc = (n_units + kClusterCtas - 1) / kClusterCtas;
+    return upc <= kMaxUnitsPerCta ? upc : 0;
+}
+
 // CSR form: indptr[bg] = sum of counts before bg; indices = valid prefixes.
 __global__ void __launch_bounds__(256)
     csr_kernel(const int32_t *__restrict__ tables, const int32_t *__restrict__ counts, int n_bg,
@@ -241,6 +388,15 @@ int launch_build_tables_bits(const uint32_t *mask, int B, int H_q, int nQ, int n
                              bool page_ids, cudaStream_t stream) {
     const int H_kv = H_q / group;
     const int nW = (nKVmax + 31) / 32;
+#if CA_BUILD_CLUSTER
+    if (const int upc = cluster_upc(nW, B * H_kv)) {
+        union_tables_cluster_kernel<true><<<dim3(kClusterCtas, B * H_kv), kClusterThreads, 0,
+                                            stream>>>(mask, H_q, nQ, nKVmax, group, upc, tables,
+                                                      counts);
+        if (cudaGetLastError() != cudaSuccess) return CA_ERR_CUDA;
+        return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
+    }
+#endif
     int wpr = ((nW + 31) / 32) * 32;
     if (wpr > kMaxThreads) wpr = kMaxThreads;
     int rg = 512 / wpr;
@@ -259,6 +415,16 @@ int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax,
                         bool page_ids, cudaStream_t stream) {
     const int H_kv = H_q / group;
     const int n_chunks = (nKVmax + 15) / 16;
+    const int vec = ((reinterpret_cast<uintptr_t>(mask) & 15u) == 0 && (nKVmax % 16) == 0) ? 1 : 0;
+#if CA_BUILD_CLUSTER
+    if (const int upc = vec ? cluster_upc(n_chunks, B * H_kv) : 0) {
+        union_tables_cluster_kernel<false><<<dim3(kClusterCtas, B * H_kv), kClusterThreads, 0,
+                                             stream>>>(mask, H_q, nQ, nKVmax, group, upc, tables,
+                                                       counts);
+        if (cudaGetLastError() != cudaSuccess) return CA_ERR_CUDA;
+        return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
+    }
+#endif
     int chp = ((n_chunks + 31) / 32) * 32;
     if (chp > kMaxThreads) chp = kMaxThreads;
     int rg = kMaxThreads / chp;
@@ -268,7 +434,6 @@ int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax,
     while (rg > 1 && chp * rg > 512) --rg;
     if (rg < 1) rg = 1;
     const int threads = chp * rg;
-    const int vec = ((reinterpret_cast<uintptr_t>(mask) & 15u) == 0 && (nKVmax % 16) == 0) ? 1 : 0;
     const size_t smem = sizeof(uint32_t) * (size_t)threads;
     union_tables_kernel<<<B * H_kv, threads, smem, stream>>>(mask, H_q, nQ, nKVmax, group, chp,
                                                               rg, vec, tables, counts);

@@ -46,6 +46,38 @@ def test_bench_tile_visible_pairs_matches_token_count():
     assert bench.tile_visible_pairs(mask, cs, C, blk) == total
 
 
+def test_bench_executed_pairs_brute_force():
+    """Executed (whole-tile) work: every packed row of an item's two tiles
+    against every key of each table block starting at or before the item's
+    last position; never below the visible pairs; equal to them when nothing
+    is causally cut (blocks wholly in the past, rows filling every tile)."""
+    rng = np.random.default_rng(6)
+    for G, C, cs in ((4, 128, (256, 64)), (8, 96, (128, 0)), (2, 256, (512, 384))):
+        B, H_kv, blk, L = 2, 2, 64, 1024
+        H_q = G * H_kv
+        nQ, nK = -(-C // blk), L // blk
+        mask = (rng.random((B, H_q, nQ, nK)) < 0.3).astype(np.uint8)
+        T, c, _, _ = oracle.block_tables(mask, G)
+        R = 128 // G
+        brute = 0
+        for b in range(B):
+            for g in range(H_kv):
+                for r0 in range(0, C, 2 * R):
+                    last = cs[b] + min(r0 + 2 * R, C) - 1
+                    for t in range(c[b, g]):
+                        if T[b, g, t] * blk <= last:
+                            brute += 2 * 128 * blk
+        ex = bench.executed_pairs(T, c, cs, C, blk, G)
+        assert ex == brute
+        assert ex >= bench.visible_pairs(T, c, cs, C, blk, G)
+    # past-only tables and full tiles: executed == visible
+    B, H_kv, G, blk, C = 1, 1, 4, 128, 256
+    T = np.array([[[0, 2, 5, -1, -1, -1, -1, -1]]], np.int32)
+    c = np.array([[3]], np.int32)
+    assert bench.executed_pairs(T, c, (768,), C, blk, G) == \
+        bench.visible_pairs(T, c, (768,), C, blk, G) == 3 * blk * C * G
+
+
 def test_pack_mask_bits_round_trip():
     """The bit-packed mask input: bit k of word w is block 32*w + k, any
     nonzero byte selects, bits past nKVmax stay clear (checked bit by bit
