@@ -213,12 +213,11 @@ __global__ void __launch_bounds__(kMaxThreads)
 // blocks of a bit mask, one 32-bit word per row). Each CTA ORs its units over
 // the group's G * nQ rows (one load per (row, unit) pair, consecutive threads
 // on consecutive units of a row, folded into shared memory by atomicOr), scans
-// its popcounts, and publishes its entry total in shared memory; after a
-// cluster barrier every CTA reads the totals of the others through
-// distributed shared memory, which gives its write offset and the table
-// length. A second cluster barrier keeps each CTA's shared memory alive until
-// the others have read it. So one (b, g) is read by kClusterCtas SMs at once
-// instead of one, and the table still comes out ascending without a sort.
+// its popcounts, and writes its entry total into every CTA's shared memory
+// (distributed shared memory stores); after one cluster barrier each CTA has
+// all the totals, which give its write offset and the table length. So one
+// (b, g) is read by kClusterCtas SMs at once instead of one, and the table
+// still comes out ascending without a sort.
 constexpr int kClusterCtas = 8;
 constexpr int kClusterThreads = 256;
 constexpr int kMaxUnitsPerCta = 1024;
@@ -233,7 +232,8 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
     __shared__ uint32_t s_bits[kMaxUnitsPerCta];
     __shared__ int s_off[kMaxUnitsPerCta];
     __shared__ int warp_sums[32];
-    __shared__ int s_total, s_base, s_n;
+    __shared__ int s_totals[kClusterCtas];  // entry totals of every CTA of the cluster
+    __shared__ int s_base, s_n;
 
     constexpr int UB = BITS ? 32 : 16;  // KV blocks per unit
     const int q = static_cast<int>(cluster.block_rank());
@@ -300,11 +300,15 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
         run += tot;
         __syncthreads();  // warp_sums is reused by the next round
     }
-    if (tid == 0) s_total = run;
+    // publish this CTA's total into slot q of every CTA of the cluster; after
+    // the barrier (release / acquire) every slot is filled and no CTA touches
+    // another's shared memory again, so none has to wait for the others to
+    // finish before it exits
+    if (tid < kClusterCtas) *cluster.map_shared_rank(&s_totals[q], tid) = run;
     cluster.sync();
     // this CTA's offset (totals of the lower ranks) and the table length
     if (tid < 32) {
-        const int t = tid < kClusterCtas ? *cluster.map_shared_rank(&s_total, tid) : 0;
+        const int t = tid < kClusterCtas ? s_totals[tid] : 0;
         int below = tid < q ? t : 0;
         int all = t;
 #pragma unroll
@@ -332,7 +336,6 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
     for (int t = n + q * kClusterThreads + tid; t < nKVmax; t += kClusterCtas * kClusterThreads)
         T[t] = -1;
     if (q == 0 && tid == 0) counts[bg] = n;
-    cluster.sync();  // the other CTAs have read s_total before anyone exits
 }
 
 // Units per CTA of the cluster form, or 0 where it does not apply. It pays
