@@ -619,8 +619,11 @@ def run_ours(args, chunks):
     # mask, queries and new K/V rows go up, O and LSE come back. The copies run
     # on two side streams and are double-buffered, so the next chunk's inputs
     # and the previous chunk's outputs cross the host link while this chunk
-    # computes; a chunk's new K/V rows are written only after the previous
-    # chunk's attention has finished reading the cache.
+    # computes. In a prefill, chunk k + 1's new K/V rows lie past every row
+    # chunk k's attention reads, so the upload of one overlaps the other;
+    # this loop repeats the same step, whose rows the previous step's
+    # attention did read, so it alternates two copies of the cache by step
+    # (the upload into a copy waits only for the last attention that read it).
     masks_h = [torch.from_numpy(m).pin_memory() for m in masks_np]
     Qs_hp = [q.pin_memory() for q in Qs_h]
     Kc_h, Vc_h = [], []
@@ -638,14 +641,18 @@ def run_ours(args, chunks):
     slot_lse = [[torch.empty_like(l) for l in LSEs] for _ in range(2)]
     slot_t = [[torch.empty_like(t) for t in tables] for _ in range(2)]
     slot_c = [[torch.empty_like(c) for c in counts] for _ in range(2)]
+    caches = [(K, V), (K.clone(), V.clone())]
+    e2e_state = {"step": 0, "cache_done": [None, None]}
 
     def e2e_run(n_steps):
         ev = lambda: torch.cuda.Event()
         comp_done = [None, None]   # last compute on each slot
         out_done = [None, None]    # last output copy from each slot
-        prev_comp = None
         h2d_stream.wait_stream(stream)
         for step in range(n_steps):
+            par = e2e_state["step"] % 2
+            e2e_state["step"] += 1
+            Kx, Vx = caches[par]
             flush.zero_()  # L2 flush between steps, on the compute stream
             for k, w in enumerate(chunks):
                 u = step * n + k
@@ -656,11 +663,11 @@ def run_ours(args, chunks):
                         h2d_stream.wait_event(comp_done[sl])
                     slot_mask[sl][k].copy_(masks_h[k], non_blocking=True)
                     slot_q[sl][k].copy_(Qs_hp[k], non_blocking=True)
-                    if prev_comp is not None:
-                        h2d_stream.wait_event(prev_comp)
+                    if k == 0 and e2e_state["cache_done"][par] is not None:
+                        h2d_stream.wait_event(e2e_state["cache_done"][par])
                     for b in range(w.B):
-                        K[b, :, cs[b]:cs[b] + w.C].copy_(Kc_h[k][b], non_blocking=True)
-                        V[b, :, cs[b]:cs[b] + w.C].copy_(Vc_h[k][b], non_blocking=True)
+                        Kx[b, :, cs[b]:cs[b] + w.C].copy_(Kc_h[k][b], non_blocking=True)
+                        Vx[b, :, cs[b]:cs[b] + w.C].copy_(Vc_h[k][b], non_blocking=True)
                     in_ready = ev()
                     in_ready.record(h2d_stream)
                 stream.wait_event(in_ready)
@@ -668,13 +675,12 @@ def run_ours(args, chunks):
                     stream.wait_event(out_done[sl])
                 ca.build_block_tables(slot_mask[sl][k], w.group, tables=slot_t[sl][k],
                                       counts=slot_c[sl][k])
-                ca.chunk_attention(slot_q[sl][k], K, V, slot_t[sl][k], slot_c[sl][k],
+                ca.chunk_attention(slot_q[sl][k], Kx, Vx, slot_t[sl][k], slot_c[sl][k],
                                    w.chunk_start, O=slot_o[sl][k], LSE=slot_lse[sl][k],
                                    workspace=ws)
                 done = ev()
                 done.record(stream)
                 comp_done[sl] = done
-                prev_comp = done
                 with torch.cuda.stream(d2h_stream):
                     d2h_stream.wait_event(done)
                     Os_h[k].copy_(slot_o[sl][k], non_blocking=True)
@@ -682,6 +688,7 @@ def run_ours(args, chunks):
                     od = ev()
                     od.record(d2h_stream)
                     out_done[sl] = od
+            e2e_state["cache_done"][par] = comp_done[(step * n + n - 1) % 2]
         for sl in range(2):
             if out_done[sl] is not None:
                 stream.wait_event(out_done[sl])
@@ -792,7 +799,11 @@ def run_ours(args, chunks):
         "e2e": {"value": world * K_ * flops / (total_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "copies": "pinned host buffers; H2D and D2H on two side streams, "
-                          "double-buffered so they overlap the previous/next chunk's compute"},
+                          "double-buffered so they overlap the previous/next chunk's compute; "
+                          "two cache copies alternate by step, so a step's new K/V rows "
+                          "upload while the previous step's attention reads the other copy "
+                          "(as a prefill's next chunk writes rows the current one does not "
+                          "read)"},
         "gpu_launches": 2 * n * K_,  # table build + attention per chunk, in the timed step
         "clocks": clocks,
     }
