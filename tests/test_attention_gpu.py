@@ -203,6 +203,34 @@ def test_full_size_sampled_rows(cuda_ok, name):
     assert torch.isfinite(O.float()).all()
 
 
+def test_long_context_1m_sampled_rows(cuda_ok):
+    """1M-token context (8192 KV blocks, 2% per-head density): GPU tables
+    bit-exact, sampled rows against the oracle, NaN in every unselected block
+    and past the sequence end never reaching O."""
+    wl = workloads.by_name("llama8b_1m_d2")
+    mask = workloads.make_mask(wl)
+    Q, K, V = workloads.make_qkv(wl)
+    T, c, _, _ = oracle.block_tables(mask, wl.group)
+    Td, cd, _, _ = ca.build_block_tables(torch.from_numpy(mask).cuda(), wl.group)
+    np.testing.assert_array_equal(Td.cpu().numpy(), T)
+    np.testing.assert_array_equal(cd.cpu().numpy(), c)
+    Kd, Vd = K.cuda(), V.cuda()
+    sel = torch.zeros((wl.B, wl.H_kv, wl.nKVmax), dtype=torch.bool)
+    for b in range(wl.B):
+        for g in range(wl.H_kv):
+            sel[b, g, torch.from_numpy(T[b, g, :c[b, g]].astype(np.int64))] = True
+    shape5 = (wl.B, wl.H_kv, wl.nKVmax, wl.blk, wl.D)
+    Kd.view(shape5)[~sel.cuda()] = float("nan")
+    Vd.view(shape5)[~sel.cuda()] = float("nan")
+    ws = ca.new_workspace(wl.B, wl.H_q, wl.H_kv, wl.C, wl.blk)
+    O, L = ca.chunk_attention(Q.cuda(), Kd, Vd, Td, cd, wl.chunk_start, workspace=ws)
+    assert ca.read_device_status(ws) == ca.CA_OK
+    rows = sample_rows(wl, n_random=256)
+    O_ref, L_ref = oracle.attention(Q, K, V, wl.chunk_start, wl.blk, T, c, rows=rows)
+    compare(O, L, O_ref, L_ref, rows=rows)
+    assert torch.isfinite(O.float()).all()
+
+
 @pytest.mark.parametrize("name", ["llama8b_32k", "llama8b_128k_d10", "batched"])
 def test_full_size_dense_sampled_rows(cuda_ok, name):
     wl = workloads.by_name(name)

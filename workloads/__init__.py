@@ -38,6 +38,7 @@ __all__ = [
     "llama8b_32k",
     "llama8b_128k",
     "batched",
+    "llama8b_1m",
     "full_prefill_chunk",
     "qwen3_30b_128k",
     "by_name",
@@ -73,6 +74,7 @@ class Workload:
     n_stripes: int = -1            # fixed stripe count (-1: derive from density)
     kv_seed: Optional[int] = None  # seed for Q/K/V if it differs from ``seed``
     stripe_base: str = "cached"    # stripe count from density x ("cached" | "visible") blocks
+    kv_kind: str = "normal"        # "normal" | "pooled" (long caches; see make_kv)
 
     @property
     def group(self) -> int:
@@ -151,6 +153,19 @@ def qwen3_30b_128k(density: float = 0.10) -> Workload:
                     seed=300 + pct, mask_kind="stripes", density=density)
 
 
+def llama8b_1m(density: float = 0.02) -> Workload:
+    """1M-token context: 1,046,528 cached tokens + a 2048-token chunk (8192
+    KV blocks), the 128K sweep's per-head mask recipe (sink + local window of
+    4 + round(density * 8176) - 5 independent stripes per head). The cache is
+    drawn with the pooled recipe of ``make_kv`` (8 GB of independent normals
+    would take minutes on the host)."""
+    pct = int(round(density * 100))
+    L = 1 << 20
+    return Workload(f"llama8b_1m_d{pct}", B=1, H_q=32, H_kv=8, D=128, blk=128, C=2048,
+                    L_max=L, chunk_start=(L - 2048,), seed=500 + pct, mask_kind="stripes",
+                    density=density, kv_kind="pooled")
+
+
 def batched() -> Workload:
     """B=4 sequences with 16K/32K/64K/96K cached tokens and a 4096-token chunk;
     per-head density U(2%, 15%); heads of a group share only half of their
@@ -181,6 +196,8 @@ def by_name(name: str) -> Workload:
         return llama8b_128k(noise=True)
     if name == "batched":
         return batched()
+    if name.startswith("llama8b_1m_d"):
+        return llama8b_1m(int(name[len("llama8b_1m_d"):]) / 100.0)
     if name.startswith("qwen3_30b_128k_d"):
         return qwen3_30b_128k(int(name[len("qwen3_30b_128k_d"):]) / 100.0)
     if name.startswith("full_prefill_c"):
@@ -278,10 +295,35 @@ def make_q(wl: Workload) -> torch.Tensor:
     return _normal_bf16(_rng(wl.seed, 1), (wl.B, wl.H_q, wl.C, wl.D))
 
 
+def _make_kv_pooled(wl: Workload, seed: int) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Long caches: every (b, g, block) takes one of 64 N(0, 1) blocks of a
+    pool (a uniform index per block, separately for K and V) plus its own
+    bias vector, N(0, 2) for K and N(0, 1) for V, shared by the block's rows;
+    a read of the wrong block still sees different values."""
+    B, H, nK, blk, D = wl.B, wl.H_kv, wl.nKVmax, wl.blk, wl.D
+    n_pool = 64
+    out = []
+    for stream, bias_sd in ((2, math.sqrt(2.0)), (4, 1.0)):
+        rng = _rng(seed, stream)
+        pool = torch.from_numpy(rng.standard_normal(size=(n_pool, blk, D), dtype=np.float32))
+        idx = torch.from_numpy(rng.integers(0, n_pool, size=(B, H, nK)))
+        bias = torch.from_numpy(
+            rng.standard_normal(size=(B, H, nK, 1, D), dtype=np.float32) * np.float32(bias_sd))
+        X = torch.empty((B, H, wl.L_max, D), dtype=torch.bfloat16)
+        for b in range(B):
+            for g in range(H):
+                X[b, g] = (pool[idx[b, g]] + bias[b, g]).reshape(nK * blk, D).to(torch.bfloat16)
+        out.append(X)
+    return out[0], out[1]
+
+
 def make_kv(wl: Workload) -> Tuple[torch.Tensor, torch.Tensor]:
     """bf16 K, V [B, H_kv, L_max, D]. K = N(0,1) + per-(b, g, block) bias
-    vector with entries N(0, 2); V = N(0, 1)."""
+    vector with entries N(0, 2); V = N(0, 1). (Long caches: the pooled recipe
+    of ``_make_kv_pooled``.)"""
     seed = wl.seed if wl.kv_seed is None else wl.kv_seed
+    if wl.kv_kind == "pooled":
+        return _make_kv_pooled(wl, seed)
     shape = (wl.B, wl.H_kv, wl.L_max, wl.D)
     rk = _rng(seed, 2)
     k = rk.standard_normal(size=shape, dtype=np.float32)
