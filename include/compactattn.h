@@ -309,9 +309,12 @@ int ca_chunk_attention_noalloc(const void *Q, const void *K, const void *V, cons
                                float *LSE, unsigned int *device_status, void *stream);
 
 /*
- * Merge of attention results over disjoint key sets (CompactAttention pages,
- * "Implementation": split-KV execution cuts one query row's attention over
- * several segments of its KV blocks and merges them by their log-sum-exp).
+ * Merge of attention results over disjoint key sets. The CompactAttention
+ * pages do not describe split-KV; this is the standard log-sum-exp identity
+ * split-KV execution rests on (one query row's attention cut over several
+ * segments of its table, each segment normalised on its own), the same one
+ * ca_chunk_attention applies inside a launch to its last-wave segments, here
+ * for results of separate calls (other tables, streams or GPUs).
  * Each part i holds, for the same query rows, O_i normalised over its own
  * keys and LSE_i = ln sum exp(score) over them (natural log, the convention of
  * ca_chunk_attention's LSE output). The merged result is attention over the

@@ -1,10 +1,10 @@
 // merge_states.cu — merge of attention results over disjoint key sets.
 //
-// Split-KV execution (the CompactAttention pages, "Implementation": the
-// attention of one query row may be cut over several segments of its KV
-// blocks) leaves, per segment i, an output O_i normalised over its own keys and
-// the log-sum-exp LSE_i of its scores. Attention over the union of the key
-// sets is then
+// Split-KV execution (not on the CompactAttention pages: the standard way to
+// spread one query row's attention over several segments of its KV blocks)
+// leaves, per segment i, an output O_i normalised over its own keys and the
+// log-sum-exp LSE_i of its scores. Attention over the union of the key sets
+// is then
 //     LSE = ln sum_i exp(LSE_i),   O = sum_i exp(LSE_i - LSE) O_i,
 // evaluated here with the largest LSE_i subtracted first. The chunk kernel
 // does this merge itself for the segments of one launch; this kernel is the
