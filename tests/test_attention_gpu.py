@@ -205,16 +205,29 @@ def test_full_size_sampled_rows(cuda_ok, name):
 
 def test_long_context_1m_sampled_rows(cuda_ok):
     """1M-token context (8192 KV blocks, 2% per-head density): GPU tables
-    bit-exact, sampled rows against the oracle, NaN in every unselected block
-    and past the sequence end never reaching O."""
+    bit-exact; the dense path on sampled rows; then, with NaN in every
+    unselected block, the table path and the paged (kv_indptr / kv_indices)
+    path on sampled rows, the poison never reaching O."""
     wl = workloads.by_name("llama8b_1m_d2")
     mask = workloads.make_mask(wl)
     Q, K, V = workloads.make_qkv(wl)
     T, c, _, _ = oracle.block_tables(mask, wl.group)
-    Td, cd, _, _ = ca.build_block_tables(torch.from_numpy(mask).cuda(), wl.group)
+    maskd = torch.from_numpy(mask).cuda()
+    Td, cd, _, _ = ca.build_block_tables(maskd, wl.group)
     np.testing.assert_array_equal(Td.cpu().numpy(), T)
     np.testing.assert_array_equal(cd.cpu().numpy(), c)
-    Kd, Vd = K.cuda(), V.cuda()
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    ws = ca.new_workspace(wl.B, wl.H_q, wl.H_kv, wl.C, wl.blk)
+    # dense: every block of the 1M cache, a few rows per group
+    Od, Ld = ca.dense_chunk_attention(Qd, Kd, Vd, wl.chunk_start, wl.blk, workspace=ws)
+    assert ca.read_device_status(ws) == ca.CA_OK
+    rng = np.random.default_rng(9)
+    rows_d = np.unique(np.concatenate([
+        [(g * wl.group * wl.C) + r for g in range(wl.H_kv) for r in (0, wl.C - 1)],
+        rng.integers(0, wl.B * wl.H_q * wl.C, size=16)]).astype(np.int64))
+    Od_ref, Ld_ref = oracle.attention(Q, K, V, wl.chunk_start, wl.blk, rows=rows_d)
+    compare(Od, Ld, Od_ref, Ld_ref, rows=rows_d)
+    # poison every block no group selected
     sel = torch.zeros((wl.B, wl.H_kv, wl.nKVmax), dtype=torch.bool)
     for b in range(wl.B):
         for g in range(wl.H_kv):
@@ -222,13 +235,17 @@ def test_long_context_1m_sampled_rows(cuda_ok):
     shape5 = (wl.B, wl.H_kv, wl.nKVmax, wl.blk, wl.D)
     Kd.view(shape5)[~sel.cuda()] = float("nan")
     Vd.view(shape5)[~sel.cuda()] = float("nan")
-    ws = ca.new_workspace(wl.B, wl.H_q, wl.H_kv, wl.C, wl.blk)
-    O, L = ca.chunk_attention(Q.cuda(), Kd, Vd, Td, cd, wl.chunk_start, workspace=ws)
-    assert ca.read_device_status(ws) == ca.CA_OK
     rows = sample_rows(wl, n_random=256)
     O_ref, L_ref = oracle.attention(Q, K, V, wl.chunk_start, wl.blk, T, c, rows=rows)
+    O, L = ca.chunk_attention(Qd, Kd, Vd, Td, cd, wl.chunk_start, workspace=ws)
+    assert ca.read_device_status(ws) == ca.CA_OK
     compare(O, L, O_ref, L_ref, rows=rows)
     assert torch.isfinite(O.float()).all()
+    ip, ix, _, _ = ca.build_kv_pages(maskd, wl.group)
+    Op, Lp = ca.paged_chunk_attention(Qd, Kd, Vd, ip, ix, wl.chunk_start, wl.blk, workspace=ws)
+    assert ca.read_device_status(ws) == ca.CA_OK
+    compare(Op, Lp, O_ref, L_ref, rows=rows)
+    assert torch.isfinite(Op.float()).all()
 
 
 @pytest.mark.parametrize("name", ["llama8b_32k", "llama8b_128k_d10", "batched"])
