@@ -57,9 +57,10 @@ __device__ __forceinline__ uint4 f32_to_bf16x8(const float (&f)[8]) {
 
 // n parts (2 <= n <= NP <= kMaxMergeParts; NP is a compile-time bound so that
 // the common two-part merge keeps few registers and many CTAs per SM).
-// vpr = D / 8 vectors per row; rpp rows per pass of the CTA. The pass loop is uniform over the CTA so that, when the
-// output LSE aliases an input LSE, a barrier separates every thread's reads of
-// the row's LSE_i from the single store of its merged LSE.
+// vpr = D / 8 vectors per row; rpp rows per pass of the CTA. The pass loop is
+// uniform over the CTA so that, when the output LSE aliases an input LSE, a
+// barrier separates every thread's reads of the row's LSE_i from the single
+// store of its merged LSE.
 template <int NP>
 __global__ void __launch_bounds__(kMergeThreads)
     merge_states_kernel(MergeParts parts, int n, long long rows, int vpr, int rpp,
