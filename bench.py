@@ -38,6 +38,12 @@ METRIC = "chunk attn ms & TFLOP/s at 128K ctx (LLaMA-8B shape); speedup vs dense
 DEFAULT_WORKLOAD = "llama8b_128k_d10"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16 tensor peak, datasheet (without 2:4 sparsity)
+# The configurations of the measurement sweep (one line each in ``configs``):
+# the small case, the 32K chunk, the 128K density sweep, the batched step and
+# the 64-chunk full prefill.
+SWEEP = ["tiny", "llama8b_32k", "llama8b_128k_d2", "llama8b_128k_d5", "llama8b_128k_d10",
+         "llama8b_128k_d20", "batched", "full_prefill"]
 PROFILES = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = [os.path.join(ROOT, "serving_block_union_b200", "csrc", f)
                   for f in ("chunk_attention.cu", "sm100_ptx.cuh")]
@@ -552,7 +558,6 @@ def run_ours(args, chunks):
     # would, so the host's per-call cost (argument checks, tensor maps) stays
     # off the device timeline instead of opening gaps between the launches.
     # Every path it is compared with gets the same treatment.
-    graphs = []
 
     def graphed(fn):
         fn()  # eager run first: one-time host set-up happens outside capture
@@ -564,8 +569,7 @@ def run_ours(args, chunks):
             with torch.cuda.graph(g, stream=side):
                 fn()
         stream.wait_stream(side)
-        graphs.append(g)
-        return g.replay
+        return g.replay  # the bound method keeps the graph alive
 
     # Merge of two attention states (split-KV across calls or GPUs): the
     # chunk's own result shape, and a large one (1M rows) whose traffic is
@@ -655,7 +659,7 @@ def run_ours(args, chunks):
     caches = [(K, V), (K.clone(), V.clone())]
     e2e_state = {"step": 0, "cache_done": [None, None]}
 
-    def e2e_run(n_steps):
+    def e2e_run(n_steps, flushed=True):
         ev = lambda: torch.cuda.Event()
         comp_done = [None, None]   # last compute on each slot
         out_done = [None, None]    # last output copy from each slot
@@ -664,10 +668,11 @@ def run_ours(args, chunks):
             par = e2e_state["step"] % 2
             e2e_state["step"] += 1
             Kx, Vx = caches[par]
-            # no L2 flush here: a step reads the other cache copy than the
-            # step before it, and the blocks it reads (185 MB at 128K / 10%)
-            # exceed the 126 MB L2, as the uploaded inputs do not stay there
-            # in a real pipeline either
+            # the same 256 MB L2 flush as the device-timed loop, on the
+            # compute stream before the step (its own time is measured below
+            # and taken out), so that no step finds its blocks in L2
+            if flushed:
+                flush.zero_()
             for k, w in enumerate(chunks):
                 u = step * n + k
                 sl = u % 2
@@ -707,14 +712,28 @@ def run_ours(args, chunks):
             if out_done[sl] is not None:
                 stream.wait_event(out_done[sl])
 
-    e2e_run(args.warmup)
+    def e2e_timed(flushed):
+        e2e_run(args.warmup, flushed)
+        barrier()
+        e_start = torch.cuda.Event(enable_timing=True)
+        e_end = torch.cuda.Event(enable_timing=True)
+        e_start.record(stream)
+        e2e_run(args.steps, flushed)
+        e_end.record(stream)
+        barrier()
+        return e_start.elapsed_time(e_end)
+
+    # time of the flush alone (median of 20), taken out of the flushed total
+    f_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(20)]
+    for a, b in f_ev:
+        a.record(stream)
+        flush.zero_()
+        b.record(stream)
     barrier()
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_start.record(stream)
-    e2e_run(args.steps)
-    e_end.record(stream)
-    barrier()
-    e2e_ms = [e_start.elapsed_time(e_end)]
+    flush_ms = statistics.median(a.elapsed_time(b) for a, b in f_ev)
+    e2e_ms = [max(e2e_timed(True) - args.steps * flush_ms, 1e-6)]
+    e2e_noflush_ms = [e2e_timed(False)]
     h2d = sum(m.numel() + 2 * q.numel() + 2 * kc.numel() + 2 * vc.numel()
               for m, q, kc, vc in zip(masks_h, Qs_hp, Kc_h, Vc_h))
     d2h = sum(2 * o.numel() + 4 * l.numel() for o, l in zip(Os_h, LSEs_h))
@@ -728,6 +747,7 @@ def run_ours(args, chunks):
     total_build = agg(build_ms)
     total_dense = agg(dense_ms)
     total_e2e = agg(e2e_ms)
+    total_e2e_noflush = agg(e2e_noflush_ms)
     total_compact = agg(compact_ms)
     total_gather = agg(gather_ms)
     total_tile = agg(tile_ms)
@@ -808,6 +828,10 @@ def run_ours(args, chunks):
                      "traffic": profiled_traffic(name) if n == 1 else None,
                      "peak_source": f"{peak_kind} bf16 burst (kernel timed alone, L2 flushed)",
                      "frac_of_sustained_peak": attn_tflops / peak_sus,
+                     "frac_of_nominal_peak": attn_tflops / NOMINAL_BF16_TFLOPS,
+                     "nominal_peak_source": "B200 datasheet dense bf16 (2.25 PFLOP/s, no "
+                                            "sparsity); frac is against the measured cuBLAS "
+                                            "burst",
                      "algorithmic_flop_per_launch": flops / n,
                      "kernel": "chunk_attn_kernel"},
         "e2e": {"value": world * K_ * flops / (total_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
@@ -817,11 +841,16 @@ def run_ours(args, chunks):
                           "two cache copies alternate by step, so a step's new K/V rows "
                           "upload while the previous step's attention reads the other copy "
                           "(as a prefill's next chunk writes rows the current one does not "
-                          "read); no L2 flush inside this loop: each step reads the other "
-                          "cache copy, whose selected blocks exceed L2"},
+                          "read); the 256 MB L2 flush before every step, as in the "
+                          "device-timed loop, its own time measured alone and taken out",
+                "flush_ms": flush_ms,
+                "no_flush_value": world * K_ * flops / (total_e2e_noflush * 1e-3) / 1e12},
         "gpu_launches": 2 * n * K_,  # table build + attention per chunk, in the timed step
         "clocks": clocks,
     }
+    if not args.no_sweep:
+        line["configs"] = run_sweep(args, dev, stream, flush, graphed, timed_round_robin, agg,
+                                    peak, gpu_index)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         last = chunks[-1]
         v, nrows, dt, threads = oracle_sample_rate(last, masks_np[-1], Qs_h[-1], Kh, Vh,
@@ -838,6 +867,104 @@ def run_ours(args, chunks):
     return 0
 
 
+def run_sweep(args, dev, stream, flush, graphed, timed_round_robin, agg, peak, gpu_index):
+    """Every configuration of the sweep, measured the way the headline is:
+    per step the table build + attention (and the dense path over the same
+    chunks), each replayed as a CUDA graph, round robin, a 256 MB L2 flush
+    before every timed call. One configuration at a time is resident.
+    Returns {name: {...}}: ms per chunk, effective TFLOP/s of the attention,
+    its fraction of the measured burst peak, union density, and speed-up of
+    the whole step over the dense path; for ``full_prefill`` the totals of
+    the 64-chunk pass."""
+    import torch
+
+    import serving_block_union_b200 as ca
+    import workloads
+
+    out = {}
+    samplers = []
+    for name in SWEEP:
+        chunks = step_chunks(name)
+        n = len(chunks)
+        wl0 = chunks[-1]
+        Kh, Vh = workloads.make_kv(wl0)
+        K, V = Kh.to(dev), Vh.to(dev)
+        del Kh, Vh
+        masks_np = [workloads.make_mask(w) for w in chunks]
+        masks = [torch.from_numpy(m).to(dev) for m in masks_np]
+        Qs = [workloads.make_q(w).to(dev) for w in chunks]
+        tables = [torch.empty((w.B, w.H_kv, w.nKVmax), dtype=torch.int32, device=dev)
+                  for w in chunks]
+        counts = [torch.empty((w.B, w.H_kv), dtype=torch.int32, device=dev) for w in chunks]
+        Os = [torch.empty_like(q) for q in Qs]
+        LSEs = [torch.empty((w.B, w.H_q, w.C), dtype=torch.float32, device=dev) for w in chunks]
+        ws = ca.new_workspace(wl0.B, wl0.H_q, wl0.H_kv, wl0.C, wl0.blk, device=dev)
+
+        def build():
+            for k in range(n):
+                ca.build_block_tables(masks[k], chunks[k].group, tables=tables[k],
+                                      counts=counts[k])
+
+        def attend():
+            for k in range(n):
+                ca.chunk_attention(Qs[k], K, V, tables[k], counts[k], chunks[k].chunk_start,
+                                   O=Os[k], LSE=LSEs[k], workspace=ws)
+
+        def step():
+            for k in range(n):
+                ca.build_block_tables(masks[k], chunks[k].group, tables=tables[k],
+                                      counts=counts[k])
+                ca.chunk_attention(Qs[k], K, V, tables[k], counts[k], chunks[k].chunk_start,
+                                   O=Os[k], LSE=LSEs[k], workspace=ws)
+
+        def dense():
+            for k in range(n):
+                ca.dense_chunk_attention(Qs[k], K, V, chunks[k].chunk_start, chunks[k].blk,
+                                         O=Os[k], LSE=LSEs[k], workspace=ws)
+
+        build()
+        torch.cuda.synchronize(dev)
+        flops = 0.0
+        union_num = union_den = 0
+        for k, w in enumerate(chunks):
+            T_np, c_np = tables[k].cpu().numpy(), counts[k].cpu().numpy()
+            nkv = [-(-(cs + w.C) // w.blk) for cs in w.chunk_start]
+            flops += 4.0 * w.D * visible_pairs(T_np, c_np, w.chunk_start, w.C, w.blk, w.group)
+            union_num += int(c_np.sum())
+            union_den += sum(nkv) * w.H_kv
+        runs = [graphed(step), graphed(attend), graphed(dense)]
+        steps = 3 if n > 1 else min(args.steps, 10)
+        with ClockSampler(gpu_index) as clk:
+            step_ms, attn_ms, dense_ms = timed_round_robin(runs, steps, 3)
+        samplers.append(clk.summary())
+        assert ca.read_device_status(ws) == ca.CA_OK, f"device status not OK ({name})"
+        t_step, t_attn, t_dense = (agg(x) / steps for x in (step_ms, attn_ms, dense_ms))
+        tf = flops / (t_attn * 1e-3) / 1e12
+        entry = {
+            "chunks": n, "union_density": union_num / union_den,
+            "effective_tflop": flops / 1e12,
+            "step_ms": t_step, "attn_ms": t_attn, "dense_ms": t_dense,
+            "attn_tflops": tf, "step_tflops": flops / (t_step * 1e-3) / 1e12,
+            "frac_of_peak": tf / peak, "speedup_vs_dense": t_dense / t_step,
+            "steps": steps,
+        }
+        if n == 1:
+            entry["ms_per_chunk"] = t_step
+        else:
+            entry["ms_per_chunk"] = t_step / n
+            entry["note"] = ("one step = all 64 chunks (table build + attention per chunk) "
+                             "as one CUDA graph; dense_ms = the dense path over the same chunks")
+        out[name] = entry
+        del K, V, masks, Qs, tables, counts, Os, LSEs, ws, runs
+        torch.cuda.empty_cache()
+    sm = [c["sm_mhz"] for c in samplers if c.get("sm_mhz")]
+    reasons = sorted({r for c in samplers for r in c.get("reasons", [])})
+    out["clocks"] = {"sm_mhz": statistics.median(sm) if sm else None,
+                     "sm_max_mhz": max((c.get("sm_max_mhz") or 0) for c in samplers) or None,
+                     "reasons": reasons}
+    return out
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -847,6 +974,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the per-configuration sweep (the headline line only)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -287,8 +287,10 @@ int ca_tile_chunk_attention(const void *Q, const void *K, const void *V, const i
  * path that must not enter the allocator). The paper has no counterpart: this
  * is a deployment convenience of this library.
  *
- * Same arguments and results as ca_chunk_attention minus the workspace; it
- * allocates nothing (no cudaMalloc / cudaFree, no allocating library call).
+ * Same arguments, results and host-side error codes as ca_chunk_attention
+ * minus the workspace (the checks run before anything is enqueued, so a
+ * rejected call touches nothing on the GPU); it allocates nothing (no
+ * cudaMalloc / cudaFree, no allocating library call).
  * The scratch it needs comes from a fixed 4096-byte array inside the library,
  * held by every GPU that loads the library until the process exits. That
  * holds the status word and header the kernels need at minimum, not the

@@ -51,8 +51,7 @@ __all__ = [
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-# CA_LIBRARY selects another build of the library (e.g. a tuning variant)
-_LIB_PATH = os.environ.get("CA_LIBRARY") or os.path.join(_HERE, "libcompactattn.so")
+_LIB_PATH = os.path.join(_HERE, "libcompactattn.so")
 _lock = threading.Lock()
 _lib = None
 
@@ -439,10 +438,13 @@ def chunk_attention_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     cs = _chunk_start_host(chunk_start, B)
-    st = load_library().ca_chunk_attention_noalloc(
-        _ptr(Q), _ptr(K), _ptr(V), _ptr(tables), _ptr(counts), cs, B, H_q, H_kv, C, L_max, D,
-        L_max // nK, float(scale), _ptr(O), _ptr(LSE), _ptr(device_status),
-        _stream_handle(stream, Q.device))
+    # the C side uses the scratch array of the current device: make Q's
+    # device current for the call, so scratch and stream belong together
+    with torch.cuda.device(Q.device):
+        st = load_library().ca_chunk_attention_noalloc(
+            _ptr(Q), _ptr(K), _ptr(V), _ptr(tables), _ptr(counts), cs, B, H_q, H_kv, C, L_max,
+            D, L_max // nK, float(scale), _ptr(O), _ptr(LSE), _ptr(device_status),
+            _stream_handle(stream, Q.device))
     _check("ca_chunk_attention_noalloc", st)
     return O, LSE
 

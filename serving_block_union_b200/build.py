@@ -44,18 +44,14 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False, defines=(), out: str = None) -> str:
-    """Compile the library; ``defines`` are extra ``NAME=VALUE`` tuning macros and
-    ``out`` an alternative output path (both for experiments with variants)."""
-    target = out or LIB
-    if not force and not defines and out is None and up_to_date():
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile the library (skipped when it is newer than every source)."""
+    if not force and up_to_date():
         return LIB
-    objdir = os.path.join(HERE, "_build" if not defines else "_build_" + "_".join(
-        d.replace("=", "") for d in defines))
+    objdir = os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
     common = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
               "-I", os.path.join(ROOT, "include"), "--expt-relaxed-constexpr"]
-    common += [f"-D{d}" for d in defines]
     if verbose:
         common += ["-Xptxas", "-v"]
     objs = []
@@ -63,10 +59,10 @@ def build(force: bool = False, verbose: bool = False, defines=(), out: str = Non
         obj = os.path.join(objdir, src.replace(".cu", ".o"))
         subprocess.check_call(common + ["-c", os.path.join(CSRC, src), "-o", obj])
         objs.append(obj)
-    tmp = target + f".tmp{os.getpid()}"
+    tmp = LIB + f".tmp{os.getpid()}"
     subprocess.check_call([nvcc(), *ARCH, "-shared", "-o", tmp, *objs])
-    os.replace(tmp, target)
-    return target
+    os.replace(tmp, LIB)
+    return LIB
 
 
 def main(argv=None) -> int:

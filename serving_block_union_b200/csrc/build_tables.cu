@@ -27,12 +27,6 @@ namespace {
 
 constexpr int kMaxThreads = 1024;
 
-// The cluster form of the union (below) is the default; 0 keeps the one-CTA-
-// per-(b, g) form for every shape.
-#ifndef CA_BUILD_CLUSTER
-#define CA_BUILD_CLUSTER 1
-#endif
-
 __device__ __forceinline__ uint32_t nonzero_nibble(uint32_t w) {
     // 4 bits: bit k = (byte k of w != 0)
     const uint32_t m = __vcmpne4(w, 0u);  // 0xFF in every nonzero byte
@@ -391,7 +385,6 @@ int launch_build_tables_bits(const uint32_t *mask, int B, int H_q, int nQ, int n
                              bool page_ids, cudaStream_t stream) {
     const int H_kv = H_q / group;
     const int nW = (nKVmax + 31) / 32;
-#if CA_BUILD_CLUSTER
     if (const int upc = cluster_upc(nW, B * H_kv)) {
         union_tables_cluster_kernel<true><<<dim3(kClusterCtas, B * H_kv), kClusterThreads, 0,
                                             stream>>>(mask, H_q, nQ, nKVmax, group, upc, tables,
@@ -399,7 +392,6 @@ int launch_build_tables_bits(const uint32_t *mask, int B, int H_q, int nQ, int n
         if (cudaGetLastError() != cudaSuccess) return CA_ERR_CUDA;
         return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
     }
-#endif
     int wpr = ((nW + 31) / 32) * 32;
     if (wpr > kMaxThreads) wpr = kMaxThreads;
     int rg = 512 / wpr;
@@ -419,7 +411,6 @@ int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax,
     const int H_kv = H_q / group;
     const int n_chunks = (nKVmax + 15) / 16;
     const int vec = ((reinterpret_cast<uintptr_t>(mask) & 15u) == 0 && (nKVmax % 16) == 0) ? 1 : 0;
-#if CA_BUILD_CLUSTER
     if (const int upc = vec ? cluster_upc(n_chunks, B * H_kv) : 0) {
         union_tables_cluster_kernel<false><<<dim3(kClusterCtas, B * H_kv), kClusterThreads, 0,
                                              stream>>>(mask, H_q, nQ, nKVmax, group, upc, tables,
@@ -427,7 +418,6 @@ int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax,
         if (cudaGetLastError() != cudaSuccess) return CA_ERR_CUDA;
         return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
     }
-#endif
     int chp = ((n_chunks + 31) / 32) * 32;
     if (chp > kMaxThreads) chp = kMaxThreads;
     int rg = kMaxThreads / chp;

@@ -69,6 +69,15 @@ int launch_tile_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, 
 
 int launch_chunk_attention(const AttnArgs &a, int mode, cudaStream_t stream);
 
+// Host-side argument checks shared by every attention entry point (dense: no
+// tables / counts; chunk_len: NULL when every chunk has C rows). Returns CA_OK
+// or the error code the entry point reports; enqueues nothing.
+int check_attention(const void *Q, const void *K, const void *V, const int32_t *tables,
+                    const int32_t *counts, bool dense, const int32_t *chunk_start, int B, int H_q,
+                    int H_kv, int C, int L_max, int D, int blk, float scale, const void *O,
+                    const float *LSE, const void *workspace, size_t workspace_bytes,
+                    const int32_t *chunk_len = nullptr);
+
 // ---- split of the last wave (split-KV with an LSE merge)
 //
 // One CTA runs one work item (two 128-row tiles against a block list) and one
@@ -91,21 +100,11 @@ struct SplitPlan {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Build-time overrides for measurements: CA_SPLIT_FORCE = S splits every
-// item outside the first full waves into S segments (1: never split);
-// CA_SPLIT_ALL = 1 splits every item (no unsplit waves).
-#ifndef CA_SPLIT_FORCE
-#define CA_SPLIT_FORCE 0
-#endif
-#ifndef CA_SPLIT_ALL
-#define CA_SPLIT_ALL 0
-#endif
-
 inline SplitPlan plan_split(int n_items, int num_sms, int D, bool allow) {
     SplitPlan p;
     p.n_items = p.n_first = n_items;
     if (!allow || num_sms <= 0 || n_items <= 0) return p;
-    const int n_first = CA_SPLIT_ALL ? 0 : (n_items / num_sms) * num_sms;
+    const int n_first = (n_items / num_sms) * num_sms;
     const int n_rest = n_items - n_first;
     if (n_rest == 0) return p;
     int best_s = 1;
@@ -118,7 +117,6 @@ inline SplitPlan plan_split(int n_items, int num_sms, int D, bool allow) {
             best_den = s;
         }
     }
-    if (CA_SPLIT_FORCE > 0) best_s = CA_SPLIT_FORCE < kMaxSplit ? CA_SPLIT_FORCE : kMaxSplit;
     if (best_s == 1) return p;
     const size_t rows = (size_t)n_rest * best_s * kRowsPerItem;
     p.n_first = n_first;

@@ -16,11 +16,15 @@ inline bool aligned(const void *p, uintptr_t a) {
 
 inline bool supported_group(int G) { return G == 1 || G == 2 || G == 4 || G == 8 || G == 16; }
 
+}  // namespace
+
+namespace ca {
+
 int check_attention(const void *Q, const void *K, const void *V, const int32_t *tables,
                     const int32_t *counts, bool dense, const int32_t *chunk_start, int B, int H_q,
                     int H_kv, int C, int L_max, int D, int blk, float scale, const void *O,
                     const float *LSE, const void *workspace, size_t workspace_bytes,
-                    const int32_t *chunk_len = nullptr) {
+                    const int32_t *chunk_len) {
     if (!Q || !K || !V || !O || !chunk_start || !workspace) return CA_ERR_INVALID_ARG;
     if (!dense && (!tables || !counts)) return CA_ERR_INVALID_ARG;
     if (B <= 0 || H_q <= 0 || H_kv <= 0 || C <= 0 || L_max <= 0 || D <= 0 || blk <= 0)
@@ -50,7 +54,9 @@ int check_attention(const void *Q, const void *K, const void *V, const int32_t *
     return CA_OK;
 }
 
-}  // namespace
+}  // namespace ca
+
+using ca::check_attention;
 
 extern "C" {
 

@@ -27,10 +27,7 @@
 // merges them (an atomic counter, no waiting).
 //
 // FP8 (template flag): E4M3 Q, K, V, kind::f8f6f4 MMAs (K = 32 per step), P
-// rounded to E4M3 as 2^(x + 8) in TMEM (four values per column). Two build
-// switches keep measured alternatives that were slower: P in shared memory
-// (CA_P_SMEM) and S in two N = 64 halves (CA_SPLIT_S); both add shared-memory
-// traffic to MMAs that already use all of its bandwidth.
+// rounded to E4M3 as 2^(x + 8) in TMEM (four values per column).
 //
 // Warp roles (384 threads, one CTA per SM):
 //   warps 0-3  softmax + epilogue of tile 0 (thread = TMEM lane = packed row)
@@ -72,33 +69,14 @@ constexpr int kTileM = 128;
 // softmax warpgroups then grow to kSoftmaxRegs and the third shrinks to
 // kControlRegs, so that per sub-partition (one warp of each warpgroup)
 // 2 * kSoftmaxRegs + kControlRegs = 3 * kLaunchRegs (208 + 208 + 88 = 504).
-// Without the split (CA_REG_SPLIT=0) the kernel runs 320 threads at 168.
-#ifndef CA_REG_SPLIT
-#define CA_REG_SPLIT 1
-#endif
-// Softmax warps per row: 1 (a thread owns a whole S row) or 2 (two warps on the
-// same TMEM lanes take one half of the row's columns each, and exchange their
-// partial row maxima and sums through shared memory).
-#ifndef CA_COL_SPLIT
-#define CA_COL_SPLIT 1
-#endif
-constexpr int kColSplit = CA_COL_SPLIT;
-static_assert(kColSplit == 1 || kColSplit == 2, "column split must be 1 or 2");
-constexpr bool kRegSplit = CA_REG_SPLIT != 0;
-constexpr int kSoftmaxWarps = 8 * kColSplit;
+constexpr int kSoftmaxWarps = 8;
 constexpr int kMmaWarp = kSoftmaxWarps;
 constexpr int kTmaWarp = kSoftmaxWarps + 1;
-// control warpgroup padded to 4 warps when the register split needs whole warpgroups
-constexpr int kThreads = 32 * (kSoftmaxWarps + (kRegSplit ? 4 : 2));
-constexpr int kLaunchRegs = kColSplit == 1 ? 168 : 96;
-#ifndef CA_SOFTMAX_REGS
-#define CA_SOFTMAX_REGS (CA_COL_SPLIT == 1 ? 208 : 104)
-#endif
-constexpr int kSoftmaxRegs = CA_SOFTMAX_REGS;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 4);
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 208;
 // per SM sub-partition: one warp of each softmax warpgroup plus one control warp
-constexpr int kControlRegs = (2 * kColSplit + 1) * kLaunchRegs - 2 * kColSplit * kSoftmaxRegs;
-static_assert(2 * kColSplit * kSoftmaxRegs + kControlRegs == (2 * kColSplit + 1) * kLaunchRegs,
-              "register split must balance");
+constexpr int kControlRegs = 3 * kLaunchRegs - 2 * kSoftmaxRegs;
 static_assert(kSoftmaxRegs % 8 == 0 && kControlRegs % 8 == 0 && kControlRegs >= 24,
               "setmaxnreg counts are multiples of 8, at least 24");
 constexpr uint32_t kTmemCols = 512;
@@ -106,45 +84,9 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr int kSmemBudget = 227 * 1024;
 constexpr int kSmemFloor = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
-
-// Keys per P chunk handed from the softmax to the P.V MMA (32, 64 or 128).
-#ifndef CA_P_CHUNK_KEYS
-#define CA_P_CHUNK_KEYS 64
-#endif
-constexpr int kPChunkKeysCfg = CA_P_CHUNK_KEYS;
-
-// Where P (the bf16 probabilities) goes between the softmax and the P.V MMA.
-// 1: shared memory (128B-swizzled, the Q tile layout; P.V reads it as an SS
-// MMA). The S columns in TMEM are free as soon as the softmax has loaded them,
-// so S(j+1) runs on the tensor core while the softmax of block j computes its
-// exponentials. 0: P overwrites S in TMEM (TS-form P.V); S(j+1) then waits
-// for P.V(j) to have read P.
-#ifndef CA_P_SMEM
-#define CA_P_SMEM 0
-#endif
-constexpr bool kPSmem = CA_P_SMEM != 0;
-static_assert(!kPSmem || kColSplit == 1, "P in shared memory needs one softmax warp per row");
-
-// Exponentials before the row max (bf16, P in TMEM): after the first block the
-// softmax starts the exponentials of block j with the running max of the
-// earlier blocks as reference and computes the block's max alongside; a max
-// that grew past the rescale threshold is taken into account for the next
-// blocks (O is rescaled before P(j+1) lands, the row sum at once). A block
-// whose max jumps by more than 2^kEarlyGuard takes the max-first path, so P
-// stays finite.
-#ifndef CA_EARLY_EXP
-#define CA_EARLY_EXP 0
-#endif
-constexpr float kEarlyGuard = 64.0f;
-
-// S(j+1) in two N = 64 halves (128-key blocks, P in TMEM): P occupies the
-// first 64 columns of S only, so the upper half (keys 64..127) is computed as
-// soon as the softmax has loaded S(j); only the lower half waits for P.V(j).
-#ifndef CA_SPLIT_S
-#define CA_SPLIT_S 0
-#endif
-static_assert(kPChunkKeysCfg == 32 || kPChunkKeysCfg == 64 || kPChunkKeysCfg == 128,
-              "P chunk must be 32, 64 or 128 keys");
+// Keys per P chunk handed from the softmax to the P.V MMA (measured: 32- and
+// 128-key chunks were slower).
+constexpr int kPChunkKeysMax = 64;
 
 struct Params {
     int B, H_q, H_kv, C, L_max, G, R, n_pairs, nKVmax;
@@ -171,34 +113,21 @@ struct Layout {
     static constexpr int kEB = F8 ? 1 : 2;           // bytes per Q / K / V element
     static constexpr int kQTile = kTileM * D * kEB;  // D*kEB/128 sub-tiles of 128 rows x 128 B
     static constexpr int kKV = BLK * D * kEB;        // D*kEB/128 sub-tiles of BLK rows x 128 B
-    // P tile (shared-memory P only): BLK/64 sub-tiles of 128 rows x 128 B
-    static constexpr int kPTile = kPSmem ? kTileM * BLK * 2 : 0;
-    static constexpr int kXchBytes = kColSplit == 2 ? 2 * 4 * 2 * 32 * 4 : 0;
-    static constexpr int kRoom = kSmemBudget - 2048 - 2 * kQTile - 2 * kPTile - kXchBytes;
-    // K and V ring stages. P in TMEM: equal rings. P in shared memory: K needs
-    // two stages (S(j+1) is issued before P.V(j)), V one fewer when short of room.
+    static constexpr int kRoom = kSmemBudget - 2048 - 2 * kQTile;
+    // K and V ring stages (equal rings): as many as fit, at most 4
     static constexpr int kFit = kRoom / kKV;  // K + V stages that fit
-    static constexpr int kStagesK = kPSmem ? (kFit >= 8 ? 4 : (kFit + 1) / 2) : (kFit / 2 > 4 ? 4 : kFit / 2);
-    static constexpr int kStagesV = kPSmem ? (kFit - kStagesK > 4 ? 4 : kFit - kStagesK) : kStagesK;
-    static constexpr int kStages = kStagesK;  // ring depth used where K and V agree
+    static constexpr int kStages = kFit / 2 > 4 ? 4 : kFit / 2;
     static constexpr int kQOff = 0;
     static constexpr int kKOff = 2 * kQTile;
-    static constexpr int kVOff = kKOff + kStagesK * kKV;
-    static constexpr int kPOff = kVOff + kStagesV * kKV;
-    static constexpr int kBarOff = kPOff + 2 * kPTile;
-    static constexpr int kPChunkKeys =
-        kColSplit == 2 ? BLK / 2 : (kPChunkKeysCfg < BLK ? kPChunkKeysCfg : BLK);
+    static constexpr int kVOff = kKOff + kStages * kKV;
+    static constexpr int kBarOff = kVOff + kStages * kKV;
+    static constexpr int kPChunkKeys = kPChunkKeysMax < BLK ? kPChunkKeysMax : BLK;
     static constexpr int kPChunks = BLK / kPChunkKeys;  // P reaches the MMA chunk by chunk
-    static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 2 + 2 * kPChunks + 2 + 1 +
-                                    8 + 2 + 2;
-    static constexpr int kXchOff = kBarOff + kNumBars * 8 + 16;  // [2][4][2][32] floats
-    static constexpr int kEnd = kXchOff + kXchBytes;
+    static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 * kPChunks + 2 + 1;
+    static constexpr int kEnd = kBarOff + kNumBars * 8 + 16;
     static constexpr int kDynamic = (kEnd + 1024) > kSmemFloor ? (kEnd + 1024) : kSmemFloor;
-    static_assert(kStagesK >= 2 && kStagesV >= 1, "need two K stages and a V stage");
-    static_assert(kPSmem || kStagesV >= 2, "need two V stages");
-    static_assert(!kPSmem || kPChunkKeys == 64, "shared-memory P hands over 64-key sub-tiles");
+    static_assert(kStages >= 2, "need two K / V stages");
     static_assert(kDynamic <= kSmemBudget, "shared memory budget exceeded");
-    static_assert(!F8 || !kPSmem, "FP8 keeps P in TMEM");
 };
 
 // KV block index of a table entry (span-table entries carry Q-block bits
@@ -226,31 +155,6 @@ __device__ __forceinline__ int count_le(const int32_t *T, int n, int bound, int 
     return 0;
 }
 
-// Share of the softmax exponentials evaluated by the FMA-pipe polynomial
-// (exp2_poly2) instead of the MUFU unit, in pairs of columns.
-#ifndef CA_POLY_EVERY
-#define CA_POLY_EVERY 0
-#endif
-constexpr int kPolyEvery = CA_POLY_EVERY;
-
-// Pair q (columns 2q, 2q+1) of an S row goes to the FMA-pipe polynomial when
-// q % kPolyEvery == kPolyEvery - 1 (0 disables it).
-__device__ __forceinline__ constexpr bool use_poly_pair(int q) {
-    return kPolyEvery > 0 && (q % kPolyEvery) == kPolyEvery - 1;
-}
-
-// Stores 64 bf16 probabilities of one row (32 packed pairs: keys 8u .. 8u+7 in
-// pk[4u .. 4u+3]) into row m of a 128-row x 128-byte sub-tile of the P tile,
-// 128B-swizzled like the TMA-loaded Q tile (16-byte unit u of row m sits at
-// unit u ^ (m & 7)), so the P.V MMA reads it with the Q tile's descriptor.
-__device__ __forceinline__ void store_p_chunk(uint8_t *subtile, int m, const uint32_t (&pk)[32]) {
-    uint8_t *row = subtile + m * 128;
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-        *reinterpret_cast<uint4 *>(row + ((u ^ (m & 7)) << 4)) =
-            make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-}
-
 // Named barrier 1 over the softmax warps only (barrier 0 is __syncthreads).
 __device__ __forceinline__ void softmax_bar_sync() {
     asm volatile("bar.sync 1, %0;" ::"n"(kSoftmaxWarps * 32) : "memory");
@@ -266,10 +170,6 @@ template <>
 __device__ __forceinline__ void tmem_ld_row<64>(uint32_t taddr, uint32_t (&r)[64]) {
     tmem_ld64(taddr, r);
 }
-template <>
-__device__ __forceinline__ void tmem_ld_row<32>(uint32_t taddr, uint32_t (&r)[32]) {
-    tmem_ld32(taddr, r);
-}
 
 template <int D, int BLK, int MODE, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -281,8 +181,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr bool COMPACT = MODE == kModeCompact;  // K/V block t sits at row t * BLK
     constexpr bool PERTILE = MODE == kModePerTile;  // one head per tile, span tables
     constexpr int NST = L::kStages;
-    constexpr int NSK = L::kStagesK;  // K ring
-    constexpr int NSV = L::kStagesV;  // V ring
     // FP8 (E4M3 Q, K, V; kind::f8f6f4 MMAs; P rounded to E4M3 in TMEM)
     constexpr int EB = L::kEB;
     constexpr int DCH = D * EB / 128;  // 128-byte sub-tiles along D
@@ -295,10 +193,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // FP8 P is 2^(x + 8) with the running max raised whenever a row max grows
     // by more than 1/2, so P <= 2^8.5 fits E4M3 (max 448) and values down to
     // 2^-17 of the row max stay representable; bf16 P is 2^x, threshold 8.
-    constexpr bool kSplitS = CA_SPLIT_S != 0 && !kPSmem && BLK == 128 && kColSplit == 1;
-    constexpr bool kEarly = CA_EARLY_EXP != 0 && !F8 && !kPSmem && kColSplit == 1;
-    constexpr uint32_t kIdescS64 =
-        F8 ? idesc_e4m3_f32(kTileM, 64, false) : idesc_bf16_f32(kTileM, 64, false);
     constexpr float kThresh = F8 ? 0.5f : kRescaleThreshold;
     constexpr float kPBias = F8 ? 8.0f : 0.0f;
     static_assert(!F8 || MODE == kModeTables || MODE == kModeDense,
@@ -312,18 +206,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::kBarOff);
     uint64_t *q_full = bars;
     uint64_t *k_full = bars + 1;
-    uint64_t *k_empty = k_full + NSK;
-    uint64_t *v_full = k_empty + NSK;
-    uint64_t *v_empty = v_full + NSV;
+    uint64_t *k_empty = k_full + NST;
+    uint64_t *v_full = k_empty + NST;
+    uint64_t *v_empty = v_full + NST;
     constexpr int NPC = L::kPChunks;
-    uint64_t *s_full = v_empty + NSV;   // [2]
-    uint64_t *p_full = s_full + 2;      // [2][NPC]: P chunk c of tile t stored in TMEM
+    uint64_t *s_full = v_empty + NST;     // [2]
+    uint64_t *p_full = s_full + 2;        // [2][NPC]: P chunk c of tile t stored in TMEM
     uint64_t *o_full = p_full + 2 * NPC;  // [2]
     uint64_t *mma_done = o_full + 2;
-    uint64_t *xch_bar = mma_done + 1;  // [2 tiles][4 quarters]: the two half-row warps meet
-    uint64_t *s_free = xch_bar + 8;     // [2] softmax has loaded S (shared-memory P)
-    uint64_t *p_free = s_free + 2;      // [2] P.V of the tile done (shared-memory P)
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(p_free + 2);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     int *abort_flag = reinterpret_cast<int *>(tmem_slot + 1);
     int *last_flag = abort_flag + 1;  // split items: this CTA merges the segments
 
@@ -362,11 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < NSK; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(k_full + s, 1);
             mbar_init(k_empty + s, 1);
-        }
-        for (int s = 0; s < NSV; ++s) {
             mbar_init(v_full + s, 1);
             mbar_init(v_empty + s, 1);
         }
@@ -376,11 +265,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(o_full + t, 1);
         }
         mbar_init(mma_done, 1);
-        for (int x = 0; x < 8; ++x) mbar_init(xch_bar + x, 2);
-        for (int t = 0; t < 2; ++t) {
-            mbar_init(s_free + t, 4);
-            mbar_init(p_free + t, 1);
-        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -440,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Role code sits inside the branch that re-sized its registers, so the
     // compiler allocates each role within its own budget.
     if (warp >= kMmaWarp) {
-      if (kRegSplit) regs_dec<kControlRegs>();
+      regs_dec<kControlRegs>();
       if (warp == kTmaWarp) {
         // ================================================================ producer
         int k_issued = 0, v_issued = 0;  // loads started (for the drain below)
@@ -454,21 +338,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     q_full, dc * XIN, r0 + t * R, b * P.H_q + head0);
             }
             q_issued = true;
-            // K(j) into ring stage j % NSK, V(j) into j % NSV (lane 0 only);
-            // false if a wait gave up
-            auto load_k = [&](int j, int blk_idx) -> bool {
-                const int s = j % NSK;
-                if (!mbar_wait(k_empty + s, ((j / NSK) & 1) ^ 1, ab)) return false;
+            // K(j) and V(j) into ring stage j % NST (lane 0 only); false if a
+            // wait gave up
+            auto load_kv = [&](int j, int blk_idx) -> bool {
+                const int s = j % NST;
+                const uint32_t par = ((j / NST) & 1) ^ 1;
+                if (!mbar_wait(k_empty + s, par, ab)) return false;
                 mbar_arrive_expect_tx(k_full + s, L::kKV);
                 for (int dc = 0; dc < DCH; ++dc)
                     tma_load_3d(smem + L::kKOff + s * L::kKV + dc * (BLK * 128), &tmK,
                                 k_full + s, dc * XIN, blk_idx * BLK, b * P.H_kv + g);
                 k_issued = j + 1;
-                return true;
-            };
-            auto load_v = [&](int j, int blk_idx) -> bool {
-                const int s = j % NSV;
-                if (!mbar_wait(v_empty + s, ((j / NSV) & 1) ^ 1, ab)) return false;
+                if (!mbar_wait(v_empty + s, par, ab)) return false;
                 mbar_arrive_expect_tx(v_full + s, L::kKV);
                 for (int dc = 0; dc < DCH; ++dc)
                     tma_load_3d(smem + L::kVOff + s * L::kKV + dc * (BLK * 128), &tmV,
@@ -477,7 +358,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             int prev_last = -1;
-            int prev_blk = 0;  // block of the previous K load (lane 0)
             bool ok = true;
             for (int w0 = 0; w0 < n_run && ok; w0 += 32) {
                 const int jj = t0 + w0 + lane;  // table index
@@ -498,19 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int j = w0 + q;
                     const int blk_idx = COMPACT ? t0 + j : __shfl_sync(0xffffffffu, jb, q);
                     int good = 1;
-                    if (lane == 0) {
-                        // with P in shared memory, K runs one block ahead of V:
-                        // S(j + 1) is issued before P.V(j)
-                        good = load_k(j, blk_idx);
-                        if (good) {
-                            if (kPSmem) {
-                                if (j > 0) good = load_v(j - 1, prev_blk);
-                            } else {
-                                good = load_v(j, blk_idx);
-                            }
-                        }
-                        prev_blk = blk_idx;
-                    }
+                    if (lane == 0) good = load_kv(j, blk_idx);
                     good = __shfl_sync(0xffffffffu, good, 0);
                     if (!good) {
                         ok = false;
@@ -518,18 +386,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (kPSmem && ok && lane == 0) load_v(n_run - 1, prev_blk);
         }
         // drain: every copy this warp started has landed before the CTA exits
         if (lane == 0) {
             if (q_issued) mbar_wait_drain(q_full, 0);
-            for (int j = k_issued > NSK ? k_issued - NSK : 0; j < k_issued; ++j)
-                mbar_wait_drain(k_full + j % NSK, (j / NSK) & 1);
-            for (int j = v_issued > NSV ? v_issued - NSV : 0; j < v_issued; ++j)
-                mbar_wait_drain(v_full + j % NSV, (j / NSV) & 1);
+            for (int j = k_issued > NST ? k_issued - NST : 0; j < k_issued; ++j)
+                mbar_wait_drain(k_full + j % NST, (j / NST) & 1);
+            for (int j = v_issued > NST ? v_issued - NST : 0; j < v_issued; ++j)
+                mbar_wait_drain(v_full + j % NST, (j / NST) & 1);
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
+      } else if (warp == kMmaWarp) {
         // ================================================================ MMA issue
         if (n_run > 0 && lane == 0) {
             // Descriptors: the high words are constant; the low words of the Q
@@ -559,23 +426,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  kk > 0 ? 1u : 0u);
                 }
             };
-            // one N = 64 half of S(t): keys 64h .. 64h + 63 of the block (rows
-            // 64h.. of every K sub-tile) into TMEM columns 64h ..
-            auto issue_s_half = [&](int t, int slot, int h) {
-                const uint32_t a0 = q_lo + t * (L::kQTile >> 4);
-                const uint32_t b0 = k_lo + slot * kStageUnits + ((h * 64 * 128) >> 4);
-#pragma unroll
-                for (int kk = 0; kk < D / KS; ++kk) {
-                    const uint32_t ao = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
-                    const uint32_t bo = ((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4;
-                    if constexpr (F8)
-                        mma_ss_w8(tmem + t * 128 + h * 64, a0 + ao, q_hi, b0 + bo, k_hi,
-                                  kIdescS64, kk > 0 ? 1u : 0u);
-                    else
-                        mma_ss_w(tmem + t * 128 + h * 64, a0 + ao, q_hi, b0 + bo, k_hi,
-                                 kIdescS64, kk > 0 ? 1u : 0u);
-                }
-            };
             // P.V of tile t, chunk by chunk as the softmax hands P over; false if a
             // wait gave up.
             auto issue_pv = [&](int t, int slot, bool acc, uint32_t par) -> bool {
@@ -601,27 +451,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 return true;
             };
-            // P.V of tile t with P read from shared memory (64-key sub-tile c of
-            // the P tile is chunk c); false if a wait gave up.
-            const uint64_t dp = sdesc_sw128(sbase + L::kPOff, 16, 1024);
-            const uint32_t p_lo = static_cast<uint32_t>(dp), p_hi = static_cast<uint32_t>(dp >> 32);
-            auto issue_pv_smem = [&](int t, int slot, bool acc, uint32_t par) -> bool {
-                const uint32_t a0 = p_lo + t * (L::kPTile >> 4);
-                const uint32_t b0 = v_lo + slot * kStageUnits;
-#pragma unroll
-                for (int c = 0; c < NPC; ++c) {
-                    if (!mbar_wait(p_full + t * NPC + c, par, ab)) return false;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 4 * c; kk < 4 * c + 4; ++kk) {
-                        const uint32_t ao = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
-                        mma_ss_w(tmem + 256 + t * 128, a0 + ao, p_hi,
-                                 b0 + ((kk * (16 * 128)) >> 4), v_hi, kIdescPV,
-                                 (acc || kk > 0) ? 1u : 0u);
-                    }
-                }
-                return true;
-            };
             bool ok = mbar_wait(q_full, 0, ab) && mbar_wait(k_full, 0, ab);
             if (ok) {
                 tc_fence_after();
@@ -631,61 +460,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_commit(s_full + 1);
                 tc_commit(k_empty + 0);
             }
-            // P in shared memory: per block j, S(j + 1) of both tiles (as soon as
-            // each tile's softmax has loaded S(j)), then P.V(j) of both tiles.
-            for (int j = 0; kPSmem && j < n_run && ok; ++j) {
-                const bool more = j + 1 < n_run;
-                if (more) {
-                    const int ks = (j + 1) % NSK;
-                    if (!(ok = mbar_wait(k_full + ks, ((j + 1) / NSK) & 1, ab))) break;
-                    if (!(ok = mbar_wait(s_free + 0, j & 1, ab))) break;
-                    tc_fence_after();
-                    issue_s(0, ks);
-                    tc_commit(s_full + 0);
-                    if (!(ok = mbar_wait(s_free + 1, j & 1, ab))) break;
-                    tc_fence_after();
-                    issue_s(1, ks);
-                    tc_commit(s_full + 1);
-                    tc_commit(k_empty + ks);
-                }
-                const int vs = j % NSV;
-                if (!(ok = mbar_wait(v_full + vs, (j / NSV) & 1, ab))) break;
-                if (!(ok = issue_pv_smem(0, vs, j > 0, j & 1))) break;
-                tc_commit(p_free + 0);
-                if (!more) tc_commit(o_full + 0);
-                if (!(ok = issue_pv_smem(1, vs, j > 0, j & 1))) break;
-                tc_commit(p_free + 1);
-                if (!more) tc_commit(o_full + 1);
-                tc_commit(v_empty + vs);
-            }
-            // Split S: per tile, S_hi(j + 1) once the softmax has loaded S(j),
-            // then P.V(j), then S_lo(j + 1) (which overwrites P's columns; the
-            // tensor core runs one CTA's MMAs in issue order).
-            for (int j = 0; kSplitS && j < n_run && ok; ++j) {
-                const int s = j % NST;
-                const bool more = j + 1 < n_run;
-                const int s1 = (j + 1) % NST;
-                if (!(ok = mbar_wait(v_full + s, (j / NST) & 1, ab))) break;
-                if (more && !(ok = mbar_wait(k_full + s1, ((j + 1) / NST) & 1, ab))) break;
-#pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    if (more) {
-                        if (!(ok = mbar_wait(s_free + t, j & 1, ab))) break;
-                        tc_fence_after();
-                        issue_s_half(t, s1, 1);
-                    }
-                    if (!(ok = issue_pv(t, s, j > 0, j & 1))) break;
-                    if (t == 1) tc_commit(v_empty + s);
-                    if (more) {
-                        issue_s_half(t, s1, 0);
-                        tc_commit(s_full + t);
-                        if (t == 1) tc_commit(k_empty + s1);
-                    } else {
-                        tc_commit(o_full + t);
-                    }
-                }
-            }
-            for (int j = 0; !kPSmem && !kSplitS && j < n_run && ok; ++j) {
+            // per block j: P.V(j) of tile 0, S(j + 1) of tile 0, P.V(j) of tile 1,
+            // S(j + 1) of tile 1 (S overwrites the P columns the P.V before it read;
+            // the tensor core runs one CTA's MMAs in issue order)
+            for (int j = 0; j < n_run && ok; ++j) {
                 const int s = j % NST;
                 const uint32_t ph = (j / NST) & 1;
                 const bool more = j + 1 < n_run;
@@ -718,15 +496,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
     } else {
-        if (kRegSplit) regs_inc<kSoftmaxRegs>();
+        regs_inc<kSoftmaxRegs>();
         // ================================================================ softmax
-        // Warp (t, hf, qw): tile t, column part hf of the S row (kColSplit parts),
-        // TMEM lanes / packed rows 32*qw .. 32*qw + 31.
-        constexpr int CW = BLK / kColSplit;   // S columns (keys) per warp
-        constexpr int DW = D / kColSplit;     // O columns per warp
-        constexpr int CPW = NPC / kColSplit;  // P chunks per warp
-        const int t = warp / (4 * kColSplit);
-        const int hf = (warp / 4) % kColSplit;
+        // Warp (t, qw): tile t, TMEM lanes / packed rows 32*qw .. 32*qw + 31.
+        const int t = warp / 4;
         const int qw = warp & 3;
         const int m = qw * 32 + lane;
         const int h_local = m / R;
@@ -739,208 +512,91 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int member_shift = kSpanEntryBits + (r / BLK - r0 / BLK);
         const uint32_t lane_base = static_cast<uint32_t>(qw * 32) << 16;
         const uint32_t tS = tmem + lane_base + t * 128;
-        const uint32_t tO = tmem + lane_base + 256 + t * 128 + hf * DW;
+        const uint32_t tO = tmem + lane_base + 256 + t * 128;
         const float sl2 = P.scale_log2;
-        // partner exchange (column split only): partial row max / sum of the
-        // other half, through shared memory and a bounded mbarrier
-        float *xch = reinterpret_cast<float *>(smem + L::kXchOff);
-        float *xch_mine = xch + ((t * 4 + qw) * 2 + hf) * 32 + lane;
-        const float *xch_other = xch + ((t * 4 + qw) * 2 + (1 - hf)) * 32 + lane;
-        uint64_t *xbar = xch_bar + t * 4 + qw;
-        uint32_t xph = 0;
-        auto exchange = [&](float mine, float &other) -> bool {
-            *xch_mine = mine;
-            __syncwarp();
-            mbar_arrive_lane0(xbar, lane);
-            const bool got = mbar_wait(xbar, xph & 1, ab);
-            ++xph;
-            if (!__all_sync(0xffffffffu, got)) return false;
-            other = *xch_other;
-            return true;
-        };
+        // Table entries the softmax needs, fetched ahead into one register per
+        // lane: the blocks that need the causal mask (at most a few: entries
+        // past n_full; lane i holds entry n_full + i), or, in the per-tile mode,
+        // a window of 32 entries of the walk (lane i holds entry t0 + w + i).
+        const int j_mask = n_full - t0;  // walk index from which blocks are masked
+        int tab_reg = 0;
+        if (!DENSE && !PERTILE) {
+            const int e = n_full + lane;
+            tab_reg = e < n_eff ? __ldg(T + e) - base : 0;
+        }
+        if (PERTILE) tab_reg = lane < n_run ? __ldg(T + t0 + lane) : 0;
 
-        float m_run = -INFINITY, l_run = 0.0f;  // l_run: this warp's columns only
-        float pend = 1.0f;  // O rescale still owed (exponentials-first blocks)
+        float m_run = -INFINITY, l_run = 0.0f;
         float lh_run = 0.0f;  // FP8: the same sum over the E4M3-rounded P
         bool ok = true;
         for (int j = 0; j < n_run; ++j) {
+            int e_j = 0;
+            if (PERTILE) {
+                e_j = __shfl_sync(0xffffffffu, tab_reg, j & 31);
+                if ((j & 31) == 31) {  // next window of 32 entries
+                    const int e = t0 + j + 1 + lane;
+                    tab_reg = e < t0 + n_run ? __ldg(T + e) : 0;
+                }
+            }
             ok = mbar_wait(s_full + t, j & 1, ab);
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            int e_j = 0;
-            if (PERTILE) e_j = __ldg(T + t0 + j);
             if (PERTILE && ((e_j >> member_shift) & 1) == 0) {
                 // block not selected by this row's Q-block: P = 0, the running
                 // max and sum are unchanged
                 uint32_t zero[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) zero[i] = 0u;
-                if constexpr (kPSmem) {
-                    // S(j) is not needed: release its columns, then zero this
-                    // row of the P tile once P.V(j - 1) has read it
+#pragma unroll
+                for (int c = 0; c < NPC; ++c) {
+                    constexpr int CK = L::kPChunkKeys;
+#pragma unroll
+                    for (int q = 0; q < CK / 32; ++q) tmem_st16(tS + c * (CK / 2) + q * 16, zero);
+                    tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
-                    mbar_arrive_lane0(s_free + t, lane);
-                    if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(p_free + t, (j - 1) & 1, ab))) {
-                        ok = false;
-                        break;
-                    }
-                    uint32_t z32[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) z32[i] = 0u;
-#pragma unroll
-                    for (int c = 0; c < NPC; ++c) {
-                        store_p_chunk(smem + L::kPOff + t * L::kPTile + c * (kTileM * 128), m, z32);
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        mbar_arrive_lane0(p_full + t * NPC + c, lane);
-                    }
-                } else {
-                    if constexpr (kSplitS) {
-                        // S(j) is not needed: its upper half can take S(j + 1)
-                        tc_fence_before();
-                        __syncwarp();
-                        mbar_arrive_lane0(s_free + t, lane);
-                    }
-#pragma unroll
-                    for (int cl = 0; cl < CPW; ++cl) {
-                        constexpr int CK = L::kPChunkKeys;
-                        const int c = hf * CPW + cl;
-#pragma unroll
-                        for (int q = 0; q < CK / 32; ++q)
-                            tmem_st16(tS + c * (CK / 2) + q * 16, zero);
-                        tmem_st_wait();
-                        tc_fence_before();
-                        __syncwarp();
-                        mbar_arrive_lane0(p_full + t * NPC + c, lane);
-                    }
+                    mbar_arrive_lane0(p_full + t * NPC + c, lane);
                 }
                 continue;
             }
-            float s[CW];
+            float s[BLK];
             {
-                uint32_t v[CW];
-                tmem_ld_row<CW>(tS + hf * CW, v);  // this warp's S columns in one round trip
+                uint32_t v[BLK];
+                tmem_ld_row<BLK>(tS, v);  // the whole S row in one round trip
 #pragma unroll
-                for (int i = 0; i < CW; ++i) s[i] = __uint_as_float(v[i]);
+                for (int i = 0; i < BLK; ++i) s[i] = __uint_as_float(v[i]);
             }
-            if constexpr (kPSmem || kSplitS) {
-                // S(j) is in registers: its TMEM columns can take S(j + 1)
-                tc_fence_before();
-                __syncwarp();
-                mbar_arrive_lane0(s_free + t, lane);
-            }
-            if (t0 + j >= n_full) {
-                int jb = DENSE ? t0 + j : (PERTILE ? block_of<true>(e_j) : __ldg(T + t0 + j) - base);
+            if (j >= j_mask) {
+                int jb = DENSE ? t0 + j
+                               : (PERTILE ? block_of<true>(e_j)
+                                          : __shfl_sync(0xffffffffu, tab_reg, (j - j_mask) & 31));
                 jb = min(max(jb, 0), P.nKVmax);  // only matters for a flagged, invalid table
-                const int lim = p - jb * BLK - hf * CW;  // columns c <= lim are visible
+                const int lim = p - jb * BLK;  // columns c <= lim are visible
 #pragma unroll
-                for (int c = 0; c < CW; ++c)
+                for (int c = 0; c < BLK; ++c)
                     if (c > lim) s[c] = -INFINITY;
             }
             // row max: 8 independent chains of 3-input max, then a short tree
-            auto row_max = [&]() -> float {
-                float mx8[8];
+            float mx8[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+            for (int k = 0; k < 8; ++k) mx8[k] = s[k];
 #pragma unroll
-                for (int c = 8; c + 8 < CW; c += 16)
+            for (int c = 8; c + 8 < BLK; c += 16)
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], s[c + k], s[c + 8 + k]);
-                if ((CW - 8) % 16 != 0) {
+                for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], s[c + k], s[c + 8 + k]);
+            if ((BLK - 8) % 16 != 0) {
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], s[CW - 8 + k]);
-                }
-                return fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
-                             fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
-            };
-            // exponentials of P chunk cl with reference m (bf16 pairs into pk, row
-            // sum into acc2)
-            auto exp_chunk = [&](int cl, float m_ref, uint32_t(&pk)[L::kPChunkKeys / 2],
-                                 uint64_t(&acc2)[4]) {
-                constexpr int CK = L::kPChunkKeys;
-                const uint64_t sl2x2 = f2_pack(sl2, sl2);
-                const uint64_t nm2 = f2_pack(-m_ref, -m_ref);
-#pragma unroll
-                for (int i = 0; i < CK / 2; ++i) {
-                    const int e0 = cl * CK + 2 * i;
-                    const uint64_t x2 = f2_fma(f2_pack(s[e0], s[e0 + 1]), sl2x2, nm2);
-                    const uint64_t p2 = f2_pack(ex2_approx(f2_lo(x2)), ex2_approx(f2_hi(x2)));
-                    acc2[i & 3] = f2_add(acc2[i & 3], p2);
-                    pk[i] = pack_bf16x2(f2_lo(p2), f2_hi(p2));
-                }
-            };
-            // hands P chunk c (in pk) to the P.V MMA through TMEM
-            auto hand_over = [&](int c, const uint32_t(&pk)[L::kPChunkKeys / 2]) {
-                constexpr int PCOLS = L::kPChunkKeys * EB / 4;
-#pragma unroll
-                for (int q = 0; q < PCOLS / 16; ++q)
-                    tmem_st16(tS + c * PCOLS + q * 16, pk + q * 16);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                mbar_arrive_lane0(p_full + t * NPC + c, lane);
-            };
-            // O *= a on the rows where a != 1 (O holds P.V up to block j - 1:
-            // S(j) was committed after that P.V was issued)
-            auto rescale_o = [&](float a) {
-#pragma unroll
-                for (int c = 0; c < DW / 16; ++c) {
-                    uint32_t v[16];
-                    tmem_ld16(tO + c * 16, v);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
-                    tmem_st16(tO + c * 16, v);
-                }
-            };
-            if constexpr (kEarly) {
-                if (__all_sync(0xffffffffu, m_run != -INFINITY)) {
-                    // exponentials first, with the running max as reference
-                    const float m_ref = m_run;
-                    uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
-                    uint32_t pk0[L::kPChunkKeys / 2];
-                    exp_chunk(0, m_ref, pk0, acc2);
-                    const float m_blk = row_max() * sl2;
-                    if (!__any_sync(0xffffffffu, m_blk > m_ref + kEarlyGuard)) {
-                        if (__any_sync(0xffffffffu, pend != 1.0f)) rescale_o(pend);
-                        pend = 1.0f;
-                        hand_over(0, pk0);
-#pragma unroll
-                        for (int cl = 1; cl < NPC; ++cl) {
-                            uint32_t pk[L::kPChunkKeys / 2];
-                            exp_chunk(cl, m_ref, pk, acc2);
-                            hand_over(cl, pk);
-                        }
-                        acc2[0] = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
-                        l_run += f2_lo(acc2[0]) + f2_hi(acc2[0]);
-                        if (m_blk > m_ref + kThresh) {  // raise the max for later blocks
-                            const float a = ex2_approx(m_ref - m_blk);
-                            l_run *= a;
-                            m_run = m_blk;
-                            pend = a;
-                        }
-                        continue;
-                    }
-                    // a jump past the guard: the max-first path below
-                }
+                for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(mx8[k], s[BLK - 8 + k]);
             }
-            float pmax = row_max();
-            if (kColSplit == 2) {
-                float other;
-                if (!exchange(pmax, other)) {
-                    ok = false;
-                    break;
-                }
-                pmax = fmaxf(pmax, other);
-            }
+            const float pmax = fmaxf(fmax3(mx8[0], mx8[1], mx8[2]),
+                                     fmax3(fmax3(mx8[3], mx8[4], mx8[5]), mx8[6], mx8[7]));
             const float m_blk = pmax * sl2;
             const float m_new = fmaxf(m_run, m_blk);
             const bool old_finite = m_run != -INFINITY;
-            const bool upd = old_finite ? (m_new > m_run + kThresh)
-                                        : (m_new != -INFINITY);
+            const bool upd = old_finite ? (m_new > m_run + kThresh) : (m_new != -INFINITY);
             float alpha = 1.0f;
             if (upd) {
                 alpha = old_finite ? ex2_approx(m_run - m_new) : 0.0f;
@@ -948,21 +604,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // O rescale (rare: only when a row's max grew past the threshold). O is
             // stable here: S(j) was committed after P.V(j-1) was issued. It must land
-            // before the first P chunk is handed over. Each warp rescales its
-            // DW columns of O.
+            // before the first P chunk is handed over.
             const bool need = upd && old_finite && j > 0;
-            // (with P in shared memory the rescale waits for P.V(j - 1) first; it
-            // runs inside the chunk loop below). A rescale still owed by an
-            // exponentials-first block is folded in.
-            if (!kPSmem && __any_sync(0xffffffffu, need || pend != 1.0f)) {
-                rescale_o((need ? alpha : 1.0f) * pend);
+            if (__any_sync(0xffffffffu, need)) {
+                const float a = need ? alpha : 1.0f;
+#pragma unroll
+                for (int c = 0; c < D / 16; ++c) {
+                    uint32_t v[16];
+                    tmem_ld16(tO + c * 16, v);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
+                    tmem_st16(tO + c * 16, v);
+                }
             }
-            pend = 1.0f;
             const float m_use = m_run == -INFINITY ? 0.0f : m_run;
             l_run *= alpha;
             // exponentials in pairs: x = s * scale_log2 - m as one f32x2 FMA, the
-            // row sum in four f32x2 accumulators; the MUFU unit does most pairs,
-            // the FMA pipe the pairs use_poly_pair() selects
+            // row sum in four f32x2 accumulators
             const uint64_t sl2x2 = f2_pack(sl2, sl2);
             const uint64_t nm2 = f2_pack(kPBias - m_use, kPBias - m_use);
             uint64_t acc2[4];
@@ -970,24 +628,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc2[k] = 0ull;
 #pragma unroll
-            for (int cl = 0; cl < CPW; ++cl) {
+            for (int c = 0; c < NPC; ++c) {
                 constexpr int CK = L::kPChunkKeys;
-                const int c = hf * CPW + cl;  // P chunk index within the row
                 constexpr int PCOLS = CK * EB / 4;  // TMEM columns of a P chunk
                 uint32_t pk[CK / 2];  // bf16 pairs; FP8: E4M3 quads in pk[0, CK/4)
                 uint64_t p_prev = 0ull;
 #pragma unroll
                 for (int i = 0; i < CK / 2; ++i) {
-                    const int e0 = cl * CK + 2 * i;  // element in this warp's s[]
+                    const int e0 = c * CK + 2 * i;
                     const uint64_t x2 = f2_fma(f2_pack(s[e0], s[e0 + 1]), sl2x2, nm2);
-                    const uint64_t p2 = use_poly_pair(c * CK / 2 + i)
-                                            ? exp2_poly2(x2)
-                                            : f2_pack(ex2_approx(f2_lo(x2)), ex2_approx(f2_hi(x2)));
+                    const uint64_t p2 = f2_pack(ex2_approx(f2_lo(x2)), ex2_approx(f2_hi(x2)));
+                    acc2[i & 3] = f2_add(acc2[i & 3], p2);
                     if constexpr (F8) {
                         // O is normalised by the sum of the E4M3 values P.V uses
                         // (an exact convex combination of V rows); the LSE keeps
                         // the fp32 sum
-                        acc2[i & 3] = f2_add(acc2[i & 3], p2);
                         if (i & 1) {
                             const uint32_t q4 = pack_e4m3x4(f2_lo(p_prev), f2_hi(p_prev),
                                                             f2_lo(p2), f2_hi(p2));
@@ -1000,52 +655,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                             p_prev = p2;
                         }
                     } else {
-                        acc2[i & 3] = f2_add(acc2[i & 3], p2);
                         pk[i] = pack_bf16x2(f2_lo(p2), f2_hi(p2));
                     }
                 }
-                if constexpr (kPSmem) {
-                    if (cl == 0 && j > 0) {
-                        // P.V(j - 1) must have read this tile's P (and finished
-                        // with O) before P(j) and any O rescale land
-                        if (!__all_sync(0xffffffffu, mbar_wait(p_free + t, (j - 1) & 1, ab))) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        if (__any_sync(0xffffffffu, need)) {
-                            const float a = need ? alpha : 1.0f;
 #pragma unroll
-                            for (int oc = 0; oc < DW / 16; ++oc) {
-                                uint32_t v[16];
-                                tmem_ld16(tO + oc * 16, v);
-#pragma unroll
-                                for (int i = 0; i < 16; ++i)
-                                    v[i] = __float_as_uint(__uint_as_float(v[i]) * a);
-                                tmem_st16(tO + oc * 16, v);
-                            }
-                            tmem_st_wait();
-                            tc_fence_before();
-                        }
-                    }
-                    store_p_chunk(smem + L::kPOff + t * L::kPTile + c * (kTileM * 128), m, pk);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    mbar_arrive_lane0(p_full + t * NPC + c, lane);
-                } else {
-#pragma unroll
-                    for (int q = 0; q < PCOLS / 16; ++q)
-                        tmem_st16(tS + c * PCOLS + q * 16, pk + q * 16);
-                    tmem_st_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    mbar_arrive_lane0(p_full + t * NPC + c, lane);
-                }
+                for (int q = 0; q < PCOLS / 16; ++q) tmem_st16(tS + c * PCOLS + q * 16, pk + q * 16);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                mbar_arrive_lane0(p_full + t * NPC + c, lane);
             }
-            if (!ok) break;
             acc2[0] = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
-            const float sum = f2_lo(acc2[0]) + f2_hi(acc2[0]);
-            l_run += sum;
+            l_run += f2_lo(acc2[0]) + f2_hi(acc2[0]);
             if constexpr (F8) {
                 acch[0] = f2_add(acch[0], acch[1]);
                 lh_run = lh_run * alpha + (f2_lo(acch[0]) + f2_hi(acch[0]));
@@ -1057,25 +678,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             have_o = __all_sync(0xffffffffu, got);
             tc_fence_after();
         }
-        if (kColSplit == 2 && have_o) {
-            float other = 0.0f;
-            if (exchange(l_run, other)) {
-                l_run += other;
-            } else {
-                have_o = false;
-            }
-        }
         const float l_o = F8 ? lh_run : l_run;  // the sum O is normalised by
-        // (pend: the last block's O rescale, owed if it raised the max)
-        const float inv_l = l_o > 0.0f ? P.o_scale * pend / l_o : 0.0f;
+        const float inv_l = l_o > 0.0f ? P.o_scale / l_o : 0.0f;
         const float lse2 = (l_run > 0.0f && have_o) ? m_run + log2f(l_run) - kPBias : -INFINITY;
-        uint16_t *orow = P.O + (((size_t)b * P.H_q + h) * P.C + r) * D + hf * DW;
-        float *lse_out = (valid && hf == 0 && P.LSE != nullptr)
-                             ? P.LSE + ((size_t)b * P.H_q + h) * P.C + r
-                             : nullptr;
+        uint16_t *orow = P.O + (((size_t)b * P.H_q + h) * P.C + r) * D;
+        float *lse_out = (valid && P.LSE != nullptr) ? P.LSE + ((size_t)b * P.H_q + h) * P.C + r
+                                                      : nullptr;
         if (nseg == 1) {
 #pragma unroll
-            for (int c = 0; c < DW / 32; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
                 uint32_t v[32];
                 if (have_o) {
                     tmem_ld32(tO + c * 32, v);
@@ -1099,12 +710,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
             // Segment of a split item: its normalised O (fp32) and base-2 LSE
             // go to the workspace, one slot row per packed row.
-            const int rest = item - P.n_first;
-            const size_t row0 = (size_t)rest * nseg * kRowsPerItem + t * 128 + m;
-            const size_t mine = row0 + (size_t)seg * kRowsPerItem;
-            float *po = P.part_o + mine * D + hf * DW;
+            // (recomputed from the block index: nothing of the item decode has
+            // to stay live across the block loop for this rare path)
+            const int kseg = (int)blockIdx.x - P.n_first;
+            const int n_rest_ = P.n_items - P.n_first;
+            const int rest = kseg % n_rest_;
+            const int seg_ = kseg / n_rest_;
+            const int m_ = (warp & 3) * 32 + lane;
+            const size_t row0 = (size_t)rest * P.split * kRowsPerItem + (warp / 4) * 128 + m_;
+            const size_t mine = row0 + (size_t)seg_ * kRowsPerItem;
+            float *po = P.part_o + mine * D;
 #pragma unroll
-            for (int c = 0; c < DW / 32; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
                 uint32_t v[32];
                 if (have_o) {
                     tmem_ld32(tO + c * 32, v);
@@ -1120,13 +737,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          __uint_as_float(v[4 * i + 2]) * inv_l,
                                          __uint_as_float(v[4 * i + 3]) * inv_l);
             }
-            if (hf == 0) P.part_lse[mine] = lse2;
+            P.part_lse[mine] = lse2;
             // publish, count this segment in, and let the item's last CTA merge
             __threadfence();
             softmax_bar_sync();
             if (threadIdx.x == 0) {
                 const unsigned prev = atomicAdd(P.counters + rest, 1u);
-                *last_flag = prev + 1 == (unsigned)nseg;
+                *last_flag = prev + 1 == (unsigned)P.split;
             }
             softmax_bar_sync();
             if (*last_flag) {
@@ -1135,7 +752,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float mx = -INFINITY;
 #pragma unroll
                 for (int sg = 0; sg < kMaxSplit; ++sg) {
-                    ls[sg] = sg < nseg ? __ldcg(P.part_lse + row0 + (size_t)sg * kRowsPerItem)
+                    ls[sg] = sg < P.split ? __ldcg(P.part_lse + row0 + (size_t)sg * kRowsPerItem)
                                        : -INFINITY;
                     mx = fmaxf(mx, ls[sg]);
                 }
@@ -1147,14 +764,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const float inv_w = wsum > 0.0f ? 1.0f / wsum : 0.0f;
 #pragma unroll
-                for (int c = 0; c < DW / 32; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
                     float acc[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-                    for (int sg = 0; sg < nseg; ++sg) {
+                    for (int sg = 0; sg < P.split; ++sg) {
                         const float w = ls[sg] * inv_w;
                         const float4 *src = reinterpret_cast<const float4 *>(
-                            P.part_o + (row0 + (size_t)sg * kRowsPerItem) * D + hf * DW + c * 32);
+                            P.part_o + (row0 + (size_t)sg * kRowsPerItem) * D + c * 32);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const float4 x = __ldcg(src + i);
@@ -1242,7 +859,7 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
         if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return CA_ERR_CUDA;
         num_regs = fa.numRegs;
     }
-    if (kRegSplit && num_regs != kLaunchRegs) return CA_ERR_UNSUPPORTED;
+    if (num_regs != kLaunchRegs) return CA_ERR_UNSUPPORTED;
 
     const int G = a.H_q / a.H_kv;
     const int pack = MODE == kModePerTile ? 1 : G;  // query heads packed into a tile

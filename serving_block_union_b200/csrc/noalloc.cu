@@ -57,7 +57,16 @@ extern "C" int ca_chunk_attention_noalloc(const void *Q, const void *K, const vo
                                           const int32_t *chunk_start, int B, int H_q, int H_kv,
                                           int C, int L_max, int D, int blk, float scale, void *O,
                                           float *LSE, unsigned int *device_status, void *stream) {
-    if (ca_workspace_bytes(B, H_q, H_kv, C, blk) == 0) return CA_ERR_INVALID_ARG;
+    // The same host checks (and error codes) as ca_chunk_attention, before
+    // anything is enqueued, so that a rejected call leaves the status word of
+    // calls still in flight alone. The checks only test the workspace
+    // pointer's alignment and size, so a 256-aligned placeholder stands in
+    // for the scratch array here (it is never dereferenced).
+    const int chk = ca::check_attention(Q, K, V, tables, counts, false, chunk_start, B, H_q, H_kv,
+                                        C, L_max, D, blk, scale, O, LSE,
+                                        reinterpret_cast<const void *>(uintptr_t{256}),
+                                        kNoAllocScratchBytes);
+    if (chk != CA_OK) return chk;
     void *scratch = nullptr;
     const int st = scratch_for_current_device(&scratch);
     if (st != CA_OK) return st;

@@ -54,25 +54,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  : "memory");
 }
 
-// Suspend-time hint (ns) of the polling loop's try_wait: the waiting thread is
-// parked until the phase completes or the hint expires instead of spinning, so
-// that waiting warps leave the issue slots of their SM sub-partition to the
-// warps sharing it. 0 uses the hardware's default limit.
-#ifndef CA_WAIT_HINT_NS
-#define CA_WAIT_HINT_NS 0
-#endif
-
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-#if CA_WAIT_HINT_NS > 0
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "n"(CA_WAIT_HINT_NS)
-        : "memory");
-#else
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -80,7 +63,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "=r"(ok)
         : "r"(bar), "r"(parity)
         : "memory");
-#endif
     return ok != 0;
 }
 
@@ -428,30 +410,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
-// 2^x on the FMA pipe, for a share of the softmax exponentials so that the
-// MUFU unit is not the only one doing them. Method: Cody-Waite style range
-// reduction x = i + f with i = round(x) (round-to-nearest through the 1.5 * 2^23
-// addition trick, so no conversion instruction is needed) and f in [-1/2, 1/2],
-// then a degree-3 polynomial 1 + c1 f + c2 f^2 + c3 f^3 fitted here as the
-// minimax (equi-oscillating) relative-error approximation of 2^f on that
-// interval by linear programming on a dense grid (max relative error 1.01e-4,
-// well under the 2^-9 rounding of the bf16 probabilities it feeds), and the
-// scale by 2^i is an integer add into the exponent field. Inputs are clamped at
-// -127, where the result is exactly +0 (p(0) = 1 and 127 is subtracted from the
-// exponent of 1.0); the softmax only feeds it x <= 8.
-__device__ __forceinline__ float exp2_poly(float x) {
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    constexpr float c1 = 0.6932829022407532f;
-    constexpr float c2 = 0.2422109693288803f;
-    constexpr float c3 = 0.055009059607982635f;
-    x = fmaxf(x, -127.0f);
-    const float t = x + kRound;
-    const float r = t - kRound;
-    const float f = x - r;
-    const float p = fmaf(fmaf(fmaf(c3, f, c2), f, c1), f, 1.0f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 // max(a, b, c) in one instruction (sm_100 three-input form).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
     float r;
@@ -481,23 +439,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     uint64_t r;
     asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
-}
-
-// exp2_poly on a pair, with the pair arithmetic in f32x2 form (same method,
-// same coefficients and the same -127 clamp as exp2_poly above).
-__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
-    const uint64_t xc = f2_pack(fmaxf(f2_lo(x2), -127.0f), fmaxf(f2_hi(x2), -127.0f));
-    const uint64_t kRound2 = f2_pack(12582912.0f, 12582912.0f);
-    const uint64_t t = f2_add(xc, kRound2);
-    const uint64_t r = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
-    const uint64_t f = f2_fma(r, f2_pack(-1.0f, -1.0f), xc);
-    uint64_t p = f2_fma(f2_pack(0.055009059607982635f, 0.055009059607982635f), f,
-                        f2_pack(0.2422109693288803f, 0.2422109693288803f));
-    p = f2_fma(p, f, f2_pack(0.6932829022407532f, 0.6932829022407532f));
-    p = f2_fma(p, f, f2_pack(1.0f, 1.0f));
-    const uint32_t lo = __float_as_uint(f2_lo(t)) * 8388608u + __float_as_uint(f2_lo(p));
-    const uint32_t hi = __float_as_uint(f2_hi(t)) * 8388608u + __float_as_uint(f2_hi(p));
-    return f2_pack(__uint_as_float(lo), __uint_as_float(hi));
 }
 
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits [0,16).

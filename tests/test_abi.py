@@ -94,6 +94,33 @@ def test_attention_host_checks(lib, kw, code):
     assert _attn(lib, **kw) == code
 
 
+@pytest.mark.parametrize("kw,code", [
+    (dict(Q=None), ca.CA_ERR_INVALID_ARG),
+    (dict(counts=None), ca.CA_ERR_INVALID_ARG),
+    (dict(C=0), ca.CA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), ca.CA_ERR_INVALID_ARG),
+    (dict(H_kv=6), ca.CA_ERR_SHAPE),          # H_q % H_kv != 0: the same code as above
+    (dict(L_max=34800), ca.CA_ERR_SHAPE),
+    (dict(cs=[33000]), ca.CA_ERR_SHAPE),
+    (dict(D=96), ca.CA_ERR_UNSUPPORTED),
+    (dict(H_q=96, H_kv=3), ca.CA_ERR_UNSUPPORTED),
+    (dict(V=A_MIS), ca.CA_ERR_ALIGN),
+    (dict(LSE=ctypes.c_void_p((1 << 20) + 2)), ca.CA_ERR_ALIGN),
+])
+def test_noalloc_host_checks_match_workspace_entry_point(lib, kw, code):
+    """The allocation-free entry point reports the same host-side error codes
+    as ca_chunk_attention, before it touches the GPU (no device needed)."""
+    a = dict(Q=A16, K=A16, V=A16, tables=A16, counts=A16, B=1, H_q=32, H_kv=8, C=2048,
+             L_max=34816, D=128, blk=128, scale=0.088, O=A16, LSE=A16, cs=[32768])
+    a.update(kw)
+    cs = (ctypes.c_int32 * len(a["cs"]))(*a["cs"])
+    st = lib.ca_chunk_attention_noalloc(a["Q"], a["K"], a["V"], a["tables"], a["counts"], cs,
+                                        a["B"], a["H_q"], a["H_kv"], a["C"], a["L_max"], a["D"],
+                                        a["blk"], a["scale"], a["O"], a["LSE"], None, None)
+    assert st == code
+    assert _attn(lib, **{k: v for k, v in kw.items()}) == code
+
+
 def test_dense_host_checks(lib):
     cs = (ctypes.c_int32 * 1)(32768)
     st = lib.ca_dense_chunk_attention(A16, A16, A16, cs, 1, 32, 8, 2048, 34816, 96, 128, 0.1,

@@ -269,6 +269,49 @@ def test_all_ones_mask_equals_dense_causal_sdpa(cfg):
     np.testing.assert_allclose(LSEd, LSEref, rtol=1e-10, atol=1e-10)
 
 
+@pytest.mark.parametrize("cfg", [
+    # B, H_q, H_kv, D, blk, C, L_max, chunk_start: starts that are not block
+    # multiples and chunk lengths that are not either
+    (2, 4, 1, 16, 8, 20, 64, (5, 37)),
+    (1, 6, 2, 8, 8, 13, 48, (27,)),
+    (3, 2, 2, 4, 4, 7, 24, (0, 1, 15)),
+])
+def test_unaligned_chunk_start_equals_causal_sdpa(cfg):
+    """Chunk starts off the block grid: the dense path covers the blocks up to
+    ceil((chunk_start + C) / blk) and the table path the selected blocks, both
+    with key k visible to row r iff k <= chunk_start + r (the bottom-right
+    causal reading). Pinned against torch's fp64 SDPA with an explicit
+    token-level mask built from the mask's blocks, not from the tables."""
+    B, H_q, H_kv, D, blk, C, L, cs = cfg
+    G = H_q // H_kv
+    nQ, nK = -(-C // blk), L // blk
+    Q, K, V = _rand_qkv(sum(cfg[:7]), B, H_q, H_kv, C, L, D)
+    scale = 1.0 / math.sqrt(D)
+    # dense: every key up to the row's own position
+    Od, LSEd = oracle.attention(Q, K, V, cs, blk, None, None, scale=scale)
+    Oref, LSEref = _sdpa_masked(Q, K, V, _causal_allowed(B, H_q, C, L, cs), scale)
+    np.testing.assert_allclose(Od, Oref, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(LSEd, LSEref, rtol=1e-10, atol=1e-10)
+    # tables from a random mask; the reference key set is the union of the
+    # group's mask rows, expanded to tokens, intersected with causality
+    rng = np.random.default_rng(sum(cfg[:7]))
+    mask = _rand_mask(rng, B, H_q, nQ, nK, 0.4)
+    mask[..., 0] = 1
+    T, cnt, _, _ = oracle.block_tables(mask, G)
+    O, LSE = oracle.attention(Q, K, V, cs, blk, T, cnt, scale=scale)
+    sel = torch.from_numpy(mask.reshape(B, H_kv, G * nQ, nK).any(axis=2))  # [B, H_kv, nK]
+    tok = sel.repeat_interleave(blk, dim=2)[:, :, :L]                    # [B, H_kv, L]
+    allowed = _causal_allowed(B, H_q, C, L, cs) & tok.repeat_interleave(G, dim=1)[:, :, None, :]
+    Oref, LSEref = _sdpa_masked(Q, K, V, allowed, scale)
+    np.testing.assert_allclose(O, Oref, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(LSE, LSEref, rtol=1e-10, atol=1e-10)
+    # with a dropped term (a key past the row's position), the pin fails
+    bad = _causal_allowed(B, H_q, C, L, [s + 1 for s in cs]) & \
+        tok.repeat_interleave(G, dim=1)[:, :, None, :]
+    Obad, _ = _sdpa_masked(Q, K, V, bad, scale)
+    assert np.abs(Obad - O).max() > 1e-3
+
+
 def test_dense_equals_sdpa_on_tiny_workload():
     wl = workloads.tiny()
     Q, K, V = workloads.make_qkv(wl)
