@@ -80,18 +80,16 @@ int check_attention(const void *Q, const void *K, const void *V, const int32_t *
 
 // ---- split of the last wave (split-KV with an LSE merge)
 //
-// One CTA (or, in the pair form, one cluster of two CTAs) runs one work item
-// and fills its SMs, so n_items items take ceil(n_items / slots) waves, slots
-// being the items resident at once, and the last wave can be mostly empty
-// (256 items on 148 SMs: 1.73 waves of work in 2). The plan keeps the full
-// waves [0, n_first) whole and cuts each remaining item's block list into
-// `split` segments run by separate CTAs (clusters), choosing the split that
-// makes those segment waves shortest. Each segment CTA writes a normalised
-// fp32 partial O and its base-2 LSE of its own rows to the workspace; the
-// last of the segment CTAs of the same rows to finish merges them (workspace
-// counters, no waiting).
+// One CTA runs one work item (two 128-row tiles against a block list) and one
+// CTA fits an SM, so n_items CTAs take ceil(n_items / SMs) waves and the last
+// wave can be mostly empty (256 items on 148 SMs: 1.73 waves of work in 2).
+// The plan keeps the full waves [0, n_first) whole and cuts each remaining
+// item's block list into `split` segments run by separate CTAs, choosing the
+// split that makes those segment waves shortest. Each segment CTA writes a
+// normalised fp32 partial O and its base-2 LSE to the workspace; the last of
+// an item's CTAs to finish merges them (workspace counters, no waiting).
 constexpr int kMaxSplit = 8;
-constexpr int kRowsPerItem = 256;     // packed rows of one CTA of an item (two tiles)
+constexpr int kRowsPerItem = 256;     // packed rows of one item (two tiles)
 constexpr int kSplitMinBlocks = 64;   // items shorter than this are not split
 
 struct SplitPlan {
@@ -102,18 +100,17 @@ struct SplitPlan {
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// ctas: CTAs per item (1, or 2 for the pair form); slots: items resident at once.
-inline SplitPlan plan_split(int n_items, int slots, int D, bool allow, int ctas = 1) {
+inline SplitPlan plan_split(int n_items, int num_sms, int D, bool allow) {
     SplitPlan p;
     p.n_items = p.n_first = n_items;
-    if (!allow || slots <= 0 || n_items <= 0) return p;
-    const int n_first = (n_items / slots) * slots;
+    if (!allow || num_sms <= 0 || n_items <= 0) return p;
+    const int n_first = (n_items / num_sms) * num_sms;
     const int n_rest = n_items - n_first;
     if (n_rest == 0) return p;
     int best_s = 1;
     long long best_waves = 1, best_den = 1;  // last waves' length as a fraction
     for (int s = 2; s <= kMaxSplit; ++s) {
-        const long long waves = ((long long)n_rest * s + slots - 1) / slots;
+        const long long waves = ((long long)n_rest * s + num_sms - 1) / num_sms;
         if (waves * best_den < best_waves * s) {  // waves / s < best
             best_s = s;
             best_waves = waves;
@@ -121,39 +118,26 @@ inline SplitPlan plan_split(int n_items, int slots, int D, bool allow, int ctas 
         }
     }
     if (best_s == 1) return p;
-    const size_t blocks = (size_t)n_rest * ctas;  // row blocks of kRowsPerItem rows
-    const size_t rows = blocks * best_s * kRowsPerItem;
+    const size_t rows = (size_t)n_rest * best_s * kRowsPerItem;
     p.n_first = n_first;
     p.split = best_s;
-    p.lse_off = kWorkspaceHeader + align256(4 * blocks);
+    p.lse_off = kWorkspaceHeader + align256(4 * (size_t)n_rest);
     p.o_off = p.lse_off + align256(4 * rows);
     p.bytes = p.o_off + 4 * rows * (size_t)D;
     return p;
 }
 
-// Work items of one attention launch: B * units * row groups, the unit a KV
-// group (G query heads packed per tile) or, in the per-tile mode, a query
-// head; a row group is two 128-row tiles (four in the pair form, whose items
-// are CTA pairs).
-inline int attention_items(int B, int H_q, int H_kv, int C, bool per_tile, bool pair = false) {
+// Work items of one attention launch: B * units * pairs, the unit a KV group
+// (G query heads packed per tile) or, in the per-tile mode, a query head.
+inline int attention_items(int B, int H_q, int H_kv, int C, bool per_tile) {
     const int pack = per_tile ? 1 : H_q / H_kv;
     const int R = 128 / pack;
-    const int per = pair ? 4 : 2;
-    const int n_groups = ((C + R - 1) / R + per - 1) / per;
-    return B * (per_tile ? H_q : H_kv) * n_groups;
-}
-
-// Whether an attention launch of this shape runs as CTA pairs.
-inline bool use_pair_form(int D, int blk, bool fp8, int mode) {
-    return !fp8 && D == 128 && blk == 128 && mode != kModePerTile;
+    const int n_pairs = ((C + R - 1) / R + 1) / 2;
+    return B * (per_tile ? H_q : H_kv) * n_pairs;
 }
 
 // SM count of the current device (cached per device; 148 if it cannot be read).
 int current_sm_count();
-
-// CTA pairs of the attention kernel resident at once on the current device
-// (cached per device; half the SM count if it cannot be read).
-int pair_slots();
 
 // Copies the K and V blocks each table selects into compact buffers: block
 // tables[b,g,t] of the cache goes to rows [t * blk, (t + 1) * blk) of Kc / Vc.

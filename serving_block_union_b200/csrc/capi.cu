@@ -82,11 +82,9 @@ size_t ca_workspace_bytes(int B, int H_q, int H_kv, int C, int blk) {
     // room for the last-wave split of either item layout, at the largest D
     const int sms = ca::current_sm_count();
     size_t bytes = ca::kWorkspaceHeader;
-    for (int form = 0; form < 3; ++form) {  // single-CTA items, per-tile items, CTA pairs
-        const bool pair = form == 2;
-        const int n = ca::attention_items(B, H_q, H_kv, C, form == 1, pair);
-        const ca::SplitPlan plan = ca::plan_split(n, pair ? ca::pair_slots() : sms, 128, true,
-                                                  pair ? 2 : 1);
+    for (int per_tile = 0; per_tile < 2; ++per_tile) {
+        const int n = ca::attention_items(B, H_q, H_kv, C, per_tile != 0);
+        const ca::SplitPlan plan = ca::plan_split(n, sms, 128, true);
         if (plan.bytes > bytes) bytes = plan.bytes;
     }
     return bytes;

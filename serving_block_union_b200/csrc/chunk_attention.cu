@@ -108,22 +108,15 @@ struct Params {
     unsigned char b_order[kMaxBatch];
 };
 
-// PAIR: the CTA is one half of a CTA pair and holds half of every K and V
-// block (keys [64 r, 64 r + 64) of K, columns [64 r, 64 r + 64) of V for
-// rank r), so a stage is half as large.
-template <int D, int BLK, bool F8 = false, bool PAIR = false>
+template <int D, int BLK, bool F8 = false>
 struct Layout {
     static constexpr int kEB = F8 ? 1 : 2;           // bytes per Q / K / V element
     static constexpr int kQTile = kTileM * D * kEB;  // D*kEB/128 sub-tiles of 128 rows x 128 B
-    // this CTA's bytes of one K (or V) block: D*kEB/128 sub-tiles of BLK rows x
-    // 128 B (pair: K in sub-tiles of BLK/2 rows, V one sub-tile of BLK rows)
-    static constexpr int kKV = BLK * D * kEB / (PAIR ? 2 : 1);
-    static constexpr int kKRows = PAIR ? BLK / 2 : BLK;  // K rows (keys) per sub-tile
+    static constexpr int kKV = BLK * D * kEB;        // D*kEB/128 sub-tiles of BLK rows x 128 B
     static constexpr int kRoom = kSmemBudget - 2048 - 2 * kQTile;
-    // K and V ring stages (equal rings): as many as fit, at most 4 (pair: 6)
+    // K and V ring stages (equal rings): as many as fit, at most 4
     static constexpr int kFit = kRoom / kKV;  // K + V stages that fit
-    static constexpr int kMaxStages = PAIR ? 6 : 4;
-    static constexpr int kStages = kFit / 2 > kMaxStages ? kMaxStages : kFit / 2;
+    static constexpr int kStages = kFit / 2 > 4 ? 4 : kFit / 2;
     static constexpr int kQOff = 0;
     static constexpr int kKOff = 2 * kQTile;
     static constexpr int kVOff = kKOff + kStages * kKV;
@@ -178,19 +171,12 @@ __device__ __forceinline__ void tmem_ld_row<64>(uint32_t taddr, uint32_t (&r)[64
     tmem_ld64(taddr, r);
 }
 
-// PAIR: launched in clusters of two CTAs that run one work item of twice the
-// rows (four 128-row tiles) as a CTA pair: both CTAs load their own Q tiles and
-// their halves of every K / V block (completions counted on the leader's
-// barriers), the leader issues cta_group::2 MMAs of M = 256 (its tile t and the
-// peer's tile t) and commits to both CTAs' barriers, and each CTA's softmax
-// works on its own tensor memory exactly as in a single CTA, handing P over on
-// the leader's barriers.
-template <int D, int BLK, int MODE, bool F8, bool PAIR>
+template <int D, int BLK, int MODE, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ Params P) {
-    using L = Layout<D, BLK, F8, PAIR>;
+    using L = Layout<D, BLK, F8>;
     constexpr bool DENSE = MODE == kModeDense;
     constexpr bool COMPACT = MODE == kModeCompact;  // K/V block t sits at row t * BLK
     constexpr bool PERTILE = MODE == kModePerTile;  // one head per tile, span tables
@@ -200,13 +186,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int DCH = D * EB / 128;  // 128-byte sub-tiles along D
     constexpr int XIN = 128 / EB;      // elements in a 128-byte sub-tile row
     constexpr int KS = 32 / EB;        // elements per MMA K step (32 bytes)
-    constexpr int MM = PAIR ? 2 * kTileM : kTileM;  // MMA rows (a pair: both CTAs' tiles)
     constexpr uint32_t kIdescS =
-        F8 ? idesc_e4m3_f32(MM, BLK, false) : idesc_bf16_f32(MM, BLK, false);
+        F8 ? idesc_e4m3_f32(kTileM, BLK, false) : idesc_bf16_f32(kTileM, BLK, false);
     constexpr uint32_t kIdescPV =
-        F8 ? idesc_e4m3_f32(MM, D, true) : idesc_bf16_f32(MM, D, true);
-    static_assert(!PAIR || (!F8 && D == 128 && BLK == 128 && MODE != kModePerTile),
-                  "the pair form runs bf16, D = 128, 128-key blocks, table / dense / compact");
+        F8 ? idesc_e4m3_f32(kTileM, D, true) : idesc_bf16_f32(kTileM, D, true);
     // FP8 P is 2^(x + 8) with the running max raised whenever a row max grows
     // by more than 1/2, so P <= 2^8.5 fits E4M3 (max 448) and values down to
     // 2^-17 of the row max stay representable; bf16 P is 2^x, threshold 8.
@@ -242,9 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the per-tile mode. CTAs [0, n_first) run items [0, n_first) whole; the
     // rest run one of `split` segments of an item's block list each
     // (segment-major, so that the CTAs resident together walk the same blocks).
-    const int rank = PAIR ? static_cast<int>(cluster_ctarank() & 1u) : 0;
-    int item = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
-    int seg = 0, nseg = 1;
+    int item = blockIdx.x, seg = 0, nseg = 1;
     if (item >= P.n_first) {
         const int k = item - P.n_first;
         const int n_rest = P.n_items - P.n_first;
@@ -263,12 +244,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int cs = P.chunk_start[b];
     const int len_b = P.chunk_len[b];  // this sequence's chunk rows
     const int R = P.R;
-    // rows of the work item: [r0c, r0c + RG); this CTA's tiles start at r0
-    const int RG = (PAIR ? 4 : 2) * R;
-    const int r0c = pair * RG;
-    const int r0 = r0c + rank * 2 * R;
-    const int r_end = min(r0c + RG, len_b);
-    const int p_min = cs + r0c;
+    const int r0 = pair * 2 * R;
+    const int r_end = min(r0 + 2 * R, len_b);
+    const int p_min = cs + r0;
     const int p_max = cs + r_end - 1;
     const int jlast = p_max / BLK;
     const int jfull = (p_min + 1) / BLK - 1;
@@ -283,8 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(s_full + t, 1);
-            // the softmax warps of both CTAs of a pair arrive on the leader's
-            for (int c = 0; c < NPC; ++c) mbar_init(p_full + t * NPC + c, PAIR ? 8 : 4);
+            for (int c = 0; c < NPC; ++c) mbar_init(p_full + t * NPC + c, 4);
             mbar_init(o_full + t, 1);
         }
         mbar_init(mma_done, 1);
@@ -297,19 +274,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tmV);
     }
     if (warp == kMmaWarp) {
-        if constexpr (PAIR) {
-            tmem_alloc_pair(tmem_slot, kTmemCols);
-            tmem_relinquish_pair();
-        } else {
-            tmem_alloc(tmem_slot, kTmemCols);
-            tmem_relinquish();
-        }
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
     }
     tc_fence_before();
-    if constexpr (PAIR)
-        cluster_sync_all();  // both CTAs' barriers exist before either uses the other's
-    else
-        __syncthreads();
+    __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const AbortState ab{abort_flag, P.status};
@@ -318,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int32_t *T = nullptr;
     int base = 0;  // paged form: entries are base + block index
     int n_eff, n_full;
-    if (r0c >= len_b) {  // an item past a shorter chunk's end: no rows, no work
+    if (r0 >= len_b) {  // a pair past a shorter chunk's end: no rows, no work
         n_eff = n_full = 0;
     } else if (DENSE) {
         n_eff = jlast + 1;
@@ -360,22 +329,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ================================================================ producer
         int k_issued = 0, v_issued = 0;  // loads started (for the drain below)
         bool q_issued = false;
-        // a pair: the leader's barriers count both CTAs' bytes; only the
-        // leader arms them, each CTA copies into its own shared memory
-        const bool arms = !PAIR || rank == 0;
-        auto lead = [&](uint64_t *bar) { return mapa_shared(smem_u32(bar), 0); };
         if (n_run > 0) {
             if (lane == 0) {
-                if (arms) mbar_arrive_expect_tx(q_full, (PAIR ? 4 : 2) * L::kQTile);
+                mbar_arrive_expect_tx(q_full, 2 * L::kQTile);
                 for (int t = 0; t < 2; ++t)
-                    for (int dc = 0; dc < DCH; ++dc) {
-                        uint8_t *dst = smem + L::kQOff + t * L::kQTile + dc * (kTileM * 128);
-                        if constexpr (PAIR)
-                            tma_load_3d_pair(dst, &tmQ, lead(q_full), dc * XIN, r0 + t * R,
-                                             b * P.H_q + head0);
-                        else
-                            tma_load_3d(dst, &tmQ, q_full, dc * XIN, r0 + t * R, b * P.H_q + head0);
-                    }
+                    for (int dc = 0; dc < DCH; ++dc)
+                        tma_load_3d(smem + L::kQOff + t * L::kQTile + dc * (kTileM * 128), &tmQ,
+                                    q_full, dc * XIN, r0 + t * R, b * P.H_q + head0);
             }
             q_issued = true;
             // K(j) and V(j) into ring stage j % NST (lane 0 only); false if a
@@ -383,28 +343,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto load_kv = [&](int j, int blk_idx) -> bool {
                 const int s = j % NST;
                 const uint32_t par = ((j / NST) & 1) ^ 1;
-                if (!mbar_wait<PAIR>(k_empty + s, par, ab)) return false;
-                if (arms) mbar_arrive_expect_tx(k_full + s, (PAIR ? 2 : 1) * L::kKV);
-                for (int dc = 0; dc < DCH; ++dc) {
-                    uint8_t *dst = smem + L::kKOff + s * L::kKV + dc * (L::kKRows * 128);
-                    if constexpr (PAIR)
-                        tma_load_3d_pair(dst, &tmK, lead(k_full + s), dc * XIN,
-                                         blk_idx * BLK + rank * (BLK / 2), b * P.H_kv + g);
-                    else
-                        tma_load_3d(dst, &tmK, k_full + s, dc * XIN, blk_idx * BLK, b * P.H_kv + g);
-                }
+                if (!mbar_wait(k_empty + s, par, ab)) return false;
+                mbar_arrive_expect_tx(k_full + s, L::kKV);
+                for (int dc = 0; dc < DCH; ++dc)
+                    tma_load_3d(smem + L::kKOff + s * L::kKV + dc * (BLK * 128), &tmK,
+                                k_full + s, dc * XIN, blk_idx * BLK, b * P.H_kv + g);
                 k_issued = j + 1;
-                if (!mbar_wait<PAIR>(v_empty + s, par, ab)) return false;
-                if (arms) mbar_arrive_expect_tx(v_full + s, (PAIR ? 2 : 1) * L::kKV);
-                if constexpr (PAIR) {
-                    // this CTA's half of the columns: one 128-byte sub-tile
-                    tma_load_3d_pair(smem + L::kVOff + s * L::kKV, &tmV, lead(v_full + s),
-                                     rank * XIN, blk_idx * BLK, b * P.H_kv + g);
-                } else {
-                    for (int dc = 0; dc < DCH; ++dc)
-                        tma_load_3d(smem + L::kVOff + s * L::kKV + dc * (BLK * 128), &tmV,
-                                    v_full + s, dc * XIN, blk_idx * BLK, b * P.H_kv + g);
-                }
+                if (!mbar_wait(v_empty + s, par, ab)) return false;
+                mbar_arrive_expect_tx(v_full + s, L::kKV);
+                for (int dc = 0; dc < DCH; ++dc)
+                    tma_load_3d(smem + L::kVOff + s * L::kKV + dc * (BLK * 128), &tmV,
+                                v_full + s, dc * XIN, blk_idx * BLK, b * P.H_kv + g);
                 v_issued = j + 1;
                 return true;
             };
@@ -439,20 +388,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         // drain: every copy this warp started has landed before the CTA exits
-        // (a pair's leader waits for both CTAs' copies, which complete on its
-        // barriers; the peer stays alive until then through the closing
-        // cluster barrier)
-        if (lane == 0 && arms) {
-            if (q_issued) mbar_wait_drain<PAIR>(q_full, 0);
+        if (lane == 0) {
+            if (q_issued) mbar_wait_drain(q_full, 0);
             for (int j = k_issued > NST ? k_issued - NST : 0; j < k_issued; ++j)
-                mbar_wait_drain<PAIR>(k_full + j % NST, (j / NST) & 1);
+                mbar_wait_drain(k_full + j % NST, (j / NST) & 1);
             for (int j = v_issued > NST ? v_issued - NST : 0; j < v_issued; ++j)
-                mbar_wait_drain<PAIR>(v_full + j % NST, (j / NST) & 1);
+                mbar_wait_drain(v_full + j % NST, (j / NST) & 1);
         }
         __syncwarp();
       } else if (warp == kMmaWarp) {
         // ================================================================ MMA issue
-        if (n_run > 0 && lane == 0 && rank == 0) {  // a pair: the leader issues
+        if (n_run > 0 && lane == 0) {
             // Descriptors: the high words are constant; the low words of the Q
             // tiles are fixed for the item and those of a K / V stage are a base
             // plus the stage offset, so each MMA costs one add and the issue.
@@ -471,11 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // 32-byte K steps (16 bf16 / 32 E4M3) inside a 128-B swizzle
                     // row; a new 128-byte sub-tile every 4 steps
                     const uint32_t ao = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
-                    const uint32_t bo = ((kk >> 2) * (L::kKRows * 128) + (kk & 3) * 32) >> 4;
-                    if constexpr (PAIR)
-                        mma_ss_pair(tmem + t * 128, a0 + ao, q_hi, b0 + bo, k_hi, kIdescS,
-                                    kk > 0 ? 1u : 0u);
-                    else if constexpr (F8)
+                    const uint32_t bo = ((kk >> 2) * (BLK * 128) + (kk & 3) * 32) >> 4;
+                    if constexpr (F8)
                         mma_ss_w8(tmem + t * 128, a0 + ao, q_hi, b0 + bo, k_hi, kIdescS,
                                   kk > 0 ? 1u : 0u);
                     else
@@ -489,18 +432,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t b0 = v_lo + slot * kStageUnits;
 #pragma unroll
                 for (int c = 0; c < NPC; ++c) {
-                    if (!mbar_wait<PAIR>(p_full + t * NPC + c, par, ab)) return false;
+                    if (!mbar_wait(p_full + t * NPC + c, par, ab)) return false;
                     tc_fence_after();
                     constexpr int KPC = L::kPChunkKeys / KS;  // MMAs (one K step each) per chunk
 #pragma unroll
                     for (int kk = KPC * c; kk < KPC * c + KPC; ++kk) {
                         // a K step is 8 TMEM columns of P (2 bf16 or 4 E4M3 per
                         // column) and KS rows of V (128 bytes per row)
-                        if constexpr (PAIR)
-                            mma_ts_pair(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
-                                        b0 + ((kk * (KS * 128)) >> 4), v_hi, kIdescPV,
-                                        (acc || kk > 0) ? 1u : 0u);
-                        else if constexpr (F8)
+                        if constexpr (F8)
                             mma_ts_w8(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
                                       b0 + ((kk * (KS * 128)) >> 4), v_hi, kIdescPV,
                                       (acc || kk > 0) ? 1u : 0u);
@@ -512,21 +451,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 return true;
             };
-            // a pair's commits arrive on the barriers of both CTAs
-            auto commit = [&](uint64_t *bar) {
-                if constexpr (PAIR)
-                    tc_commit_pair_both(bar);
-                else
-                    tc_commit(bar);
-            };
-            bool ok = mbar_wait<PAIR>(q_full, 0, ab) && mbar_wait<PAIR>(k_full, 0, ab);
+            bool ok = mbar_wait(q_full, 0, ab) && mbar_wait(k_full, 0, ab);
             if (ok) {
                 tc_fence_after();
                 issue_s(0, 0);
-                commit(s_full + 0);
+                tc_commit(s_full + 0);
                 issue_s(1, 0);
-                commit(s_full + 1);
-                commit(k_empty + 0);
+                tc_commit(s_full + 1);
+                tc_commit(k_empty + 0);
             }
             // per block j: P.V(j) of tile 0, S(j + 1) of tile 0, P.V(j) of tile 1,
             // S(j + 1) of tile 1 (S overwrites the P columns the P.V before it read;
@@ -537,32 +469,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool more = j + 1 < n_run;
                 const int s1 = (j + 1) % NST;
                 const uint32_t ph1 = ((j + 1) / NST) & 1;
-                if (!(ok = mbar_wait<PAIR>(v_full + s, ph, ab))) break;
+                if (!(ok = mbar_wait(v_full + s, ph, ab))) break;
                 if (!(ok = issue_pv(0, s, j > 0, j & 1))) break;
                 if (more) {
-                    if (!(ok = mbar_wait<PAIR>(k_full + s1, ph1, ab))) break;
+                    if (!(ok = mbar_wait(k_full + s1, ph1, ab))) break;
                     tc_fence_after();
                     issue_s(0, s1);
-                    commit(s_full + 0);
+                    tc_commit(s_full + 0);
                 } else {
-                    commit(o_full + 0);
+                    tc_commit(o_full + 0);
                 }
                 if (!(ok = issue_pv(1, s, j > 0, j & 1))) break;
-                commit(v_empty + s);
+                tc_commit(v_empty + s);
                 if (more) {
                     issue_s(1, s1);
-                    commit(s_full + 1);
-                    commit(k_empty + s1);
+                    tc_commit(s_full + 1);
+                    tc_commit(k_empty + s1);
                 } else {
-                    commit(o_full + 1);
+                    tc_commit(o_full + 1);
                 }
             }
             // drain: all MMAs issued by this thread have completed
-            if constexpr (PAIR)
-                tc_commit_pair_local(mma_done);
-            else
-                tc_commit(mma_done);
-            mbar_wait_drain<PAIR>(mma_done, 0);
+            tc_commit(mma_done);
+            mbar_wait_drain(mma_done, 0);
         }
         __syncwarp();
       }
@@ -585,16 +514,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tS = tmem + lane_base + t * 128;
         const uint32_t tO = tmem + lane_base + 256 + t * 128;
         const float sl2 = P.scale_log2;
-        // where P chunk c of this tile is announced: the leader's barrier (in a
-        // pair, the leader's MMA reads both CTAs' P)
-        const uint32_t p_full_at = PAIR ? mapa_shared(smem_u32(p_full + t * NPC), 0)
-                                        : smem_u32(p_full + t * NPC);
-        auto p_ready = [&](int c) {
-            if constexpr (PAIR)
-                mbar_arrive_cluster_lane0(p_full_at + 8 * c, lane);
-            else
-                mbar_arrive_lane0(p_full + t * NPC + c, lane);
-        };
         // Table entries the softmax needs, fetched ahead into one register per
         // lane: the blocks that need the causal mask (at most a few: entries
         // past n_full; lane i holds entry n_full + i), or, in the per-tile mode,
@@ -619,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tab_reg = e < t0 + n_run ? __ldg(T + e) : 0;
                 }
             }
-            ok = mbar_wait<PAIR>(s_full + t, j & 1, ab);
+            ok = mbar_wait(s_full + t, j & 1, ab);
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
                 break;
@@ -639,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
-                    p_ready(c);
+                    mbar_arrive_lane0(p_full + t * NPC + c, lane);
                 }
                 continue;
             }
@@ -705,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t sl2x2 = f2_pack(sl2, sl2);
             const uint64_t nm2 = f2_pack(kPBias - m_use, kPBias - m_use);
             uint64_t acc2[4];
-            uint64_t acch[2] = {0ull, 0ull};  // FP8: sums of the rounded P
+            float acch[2] = {0.0f, 0.0f};  // FP8: sums of the rounded P
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc2[k] = 0ull;
 #pragma unroll
@@ -728,10 +647,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint32_t q4 = pack_e4m3x4(f2_lo(p_prev), f2_hi(p_prev),
                                                             f2_lo(p2), f2_hi(p2));
                             pk[i >> 1] = q4;
-                            acch[(i >> 1) & 1] = f2_add(
-                                acch[(i >> 1) & 1],
-                                f2_add(e4m3x2_to_f32x2(static_cast<uint16_t>(q4)),
-                                       e4m3x2_to_f32x2(static_cast<uint16_t>(q4 >> 16))));
+                            acc_e4m3x4(q4, acch[0], acch[1]);
                         } else {
                             p_prev = p2;
                         }
@@ -744,18 +660,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                p_ready(c);
+                mbar_arrive_lane0(p_full + t * NPC + c, lane);
             }
             acc2[0] = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
             l_run += f2_lo(acc2[0]) + f2_hi(acc2[0]);
-            if constexpr (F8) {
-                acch[0] = f2_add(acch[0], acch[1]);
-                lh_run = lh_run * alpha + (f2_lo(acch[0]) + f2_hi(acch[0]));
-            }
+            if constexpr (F8) lh_run = lh_run * alpha + (acch[0] + acch[1]);
         }
         bool have_o = false;
         if (n_run > 0 && __all_sync(0xffffffffu, ok)) {
-            const bool got = mbar_wait<PAIR>(o_full + t, 0, ab);
+            const bool got = mbar_wait(o_full + t, 0, ab);
             have_o = __all_sync(0xffffffffu, got);
             tc_fence_after();
         }
@@ -793,10 +706,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // go to the workspace, one slot row per packed row.
             // (recomputed from the block index: nothing of the item decode has
             // to stay live across the block loop for this rare path)
-            const int kseg = (PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x) - P.n_first;
+            const int kseg = (int)blockIdx.x - P.n_first;
             const int n_rest_ = P.n_items - P.n_first;
-            // the rows of one CTA of an item (a pair: of one of its two CTAs)
-            const int rest = (kseg % n_rest_) * (PAIR ? 2 : 1) + rank;
+            const int rest = kseg % n_rest_;
             const int seg_ = kseg / n_rest_;
             const int m_ = (warp & 3) * 32 + lane;
             const size_t row0 = (size_t)rest * P.split * kRowsPerItem + (warp / 4) * 128 + m_;
@@ -880,29 +792,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     tc_fence_before();
-    if constexpr (PAIR) {
-        // After a bounded wait gave up, this CTA's copies may still be in
-        // flight towards its shared memory with nothing left to wait on here
-        // (a pair's copies complete on the leader's barriers): give them time
-        // to land before the CTA ends. No other path comes here early.
-        if (*abort_flag) {
-            const long long t_end = clock64() + 200000;
-            while (clock64() < t_end) {
-            }
-        }
-        // the leader's MMAs read this CTA's shared and tensor memory until its
-        // last commit: neither CTA ends (or frees TMEM) before both are done
-        cluster_sync_all();
-        if (warp == kMmaWarp) {
-            tc_fence_after();
-            tmem_dealloc_pair(tmem, kTmemCols);
-        }
-    } else {
-        __syncthreads();
-        if (warp == kMmaWarp) {
-            tc_fence_after();
-            tmem_dealloc(tmem, kTmemCols);
-        }
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -940,10 +833,10 @@ bool encode_3d(CUtensorMap *map, const void *base, int eb, uint64_t d0, uint64_t
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int BLK, int MODE, bool F8 = false, bool PAIR = false>
+template <int D, int BLK, int MODE, bool F8 = false>
 int launch_t(const AttnArgs &a, cudaStream_t stream) {
-    using L = Layout<D, BLK, F8, PAIR>;
-    auto kern = chunk_attn_kernel<D, BLK, MODE, F8, PAIR>;
+    using L = Layout<D, BLK, F8>;
+    auto kern = chunk_attn_kernel<D, BLK, MODE, F8>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -966,16 +859,15 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
     const int pack = MODE == kModePerTile ? 1 : G;  // query heads packed into a tile
     const int R = kTileM / pack;
     const int n_tiles = (a.C + R - 1) / R;
-    const int per = PAIR ? 4 : 2;  // tiles of one work item
-    const int n_pairs = (n_tiles + per - 1) / per;
+    const int n_pairs = (n_tiles + 1) / 2;
 
     constexpr int EB = L::kEB;
     constexpr uint32_t XIN = 128 / EB;  // box width: one 128-byte swizzle row
     CUtensorMap tq, tk, tv;
     if (!encode_3d(&tq, a.Q, EB, (uint64_t)D, (uint64_t)a.C, (uint64_t)a.B * a.H_q, XIN, R,
                    pack) ||
-        !encode_3d(&tk, a.K, EB, (uint64_t)D, (uint64_t)a.L_max, (uint64_t)a.B * a.H_kv, XIN,
-                   L::kKRows, 1) ||
+        !encode_3d(&tk, a.K, EB, (uint64_t)D, (uint64_t)a.L_max, (uint64_t)a.B * a.H_kv, XIN, BLK,
+                   1) ||
         !encode_3d(&tv, a.V, EB, (uint64_t)D, (uint64_t)a.L_max, (uint64_t)a.B * a.H_kv, XIN, BLK,
                    1))
         return CA_ERR_CUDA;
@@ -1027,9 +919,8 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
         alike = alike && a.chunk_start[i] == a.chunk_start[0] && len_of(i) == len_of(0);
         nkv_max = max(nkv_max, (a.chunk_start[i] + len_of(i) + BLK - 1) / BLK);
     }
-    const int ctas = PAIR ? 2 : 1;
-    SplitPlan plan = plan_split(n_items, PAIR ? pair_slots() : current_sm_count(), D,
-                                alike && nkv_max >= kSplitMinBlocks, ctas);
+    SplitPlan plan = plan_split(n_items, current_sm_count(), D,
+                                alike && nkv_max >= kSplitMinBlocks);
     if (plan.split > 1 && a.workspace_bytes < plan.bytes)
         plan = plan_split(n_items, 0, D, false);  // workspace too small: no split
     unsigned char *ws = static_cast<unsigned char *>(a.workspace);
@@ -1039,27 +930,10 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
     P.counters = reinterpret_cast<unsigned int *>(ws + kWorkspaceHeader);
     P.part_lse = reinterpret_cast<float *>(ws + plan.lse_off);
     P.part_o = reinterpret_cast<float *>(ws + plan.o_off);
-    const unsigned grid = static_cast<unsigned>(ctas * (plan.n_first +
-                                                        (n_items - plan.n_first) * plan.split));
-    if constexpr (PAIR) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(grid, 1, 1);
-        cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = L::kDynamic;
-        cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, P) != cudaSuccess) return CA_ERR_CUDA;
-        return cudaGetLastError() == cudaSuccess ? CA_OK : CA_ERR_CUDA;
-    } else {
-        kern<<<grid, kThreads, L::kDynamic, stream>>>(tq, tk, tv, P);
-        return cudaGetLastError() == cudaSuccess ? CA_OK : CA_ERR_CUDA;
-    }
+    const unsigned grid = static_cast<unsigned>(plan.n_first +
+                                                (n_items - plan.n_first) * plan.split);
+    kern<<<grid, kThreads, L::kDynamic, stream>>>(tq, tk, tv, P);
+    return cudaGetLastError() == cudaSuccess ? CA_OK : CA_ERR_CUDA;
 }
 
 }  // namespace
@@ -1080,36 +954,6 @@ int current_sm_count() {
     return cache[dev];
 }
 
-int pair_slots() {
-    static std::mutex mu;
-    static int cache[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return current_sm_count() / 2;
-    std::lock_guard<std::mutex> lock(mu);
-    if (cache[dev] == 0) {
-        using L = Layout<128, 128, false, true>;
-        auto kern = chunk_attn_kernel<128, 128, kModeTables, false, true>;
-        int n = 0;
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(2, 1, 1);
-        cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = L::kDynamic;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 L::kDynamic) != cudaSuccess ||
-            cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0)
-            n = current_sm_count() / 2;
-        cache[dev] = n;
-    }
-    return cache[dev];
-}
-
 int launch_chunk_attention(const AttnArgs &a, int mode, cudaStream_t stream) {
     if (a.fp8) {
         if (a.D != 128 || (mode != kModeTables && mode != kModeDense)) return CA_ERR_UNSUPPORTED;
@@ -1122,11 +966,6 @@ int launch_chunk_attention(const AttnArgs &a, int mode, cudaStream_t stream) {
                          : launch_t<128, 64, kModeTables, true>(a, stream);
         return CA_ERR_UNSUPPORTED;
     }
-    if (use_pair_form(a.D, a.blk, false, mode)) {  // bf16, D = 128, 128-key blocks
-        if (mode == kModeDense) return launch_t<128, 128, kModeDense, false, true>(a, stream);
-        if (mode == kModeCompact) return launch_t<128, 128, kModeCompact, false, true>(a, stream);
-        return launch_t<128, 128, kModeTables, false, true>(a, stream);
-    }
 #define CA_DISPATCH(D_, BLK_)                                                         \
     if (a.D == D_ && a.blk == BLK_) {                                                 \
         if (mode == kModeDense) return launch_t<D_, BLK_, kModeDense>(a, stream);     \
@@ -1134,8 +973,7 @@ int launch_chunk_attention(const AttnArgs &a, int mode, cudaStream_t stream) {
         if (mode == kModePerTile) return launch_t<D_, BLK_, kModePerTile>(a, stream); \
         return launch_t<D_, BLK_, kModeTables>(a, stream);                            \
     }
-    if (a.D == 128 && a.blk == 128 && mode == kModePerTile)
-        return launch_t<128, 128, kModePerTile>(a, stream);
+    CA_DISPATCH(128, 128)
     CA_DISPATCH(128, 64)
     CA_DISPATCH(64, 128)
     CA_DISPATCH(64, 64)

@@ -66,20 +66,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// The same test with acquire semantics at cluster scope: for barriers that a
-// thread of the peer CTA of a CTA pair (or a commit issued there) arrives on.
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // Shared abort state of one CTA: set once any bounded wait expires, after
 // which every other wait of the CTA returns false at once.
 struct AbortState {
@@ -90,18 +76,13 @@ struct AbortState {
 // Waits until the phase with the given parity of `bar` has completed.
 // Returns false (and records kDevErrTimeout) if the wait exceeded the limit or
 // the CTA is aborting.
-// CLUSTER: acquire at cluster scope (barriers the peer CTA of a pair arrives on).
-template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const AbortState &ab,
                                           long long limit_cycles = kWaitLimitCycles) {
     const uint32_t a = smem_u32(bar);
-    auto test = [&]() {
-        return CLUSTER ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity);
-    };
-    if (test()) return true;
+    if (mbar_try_wait(a, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-        if (test()) return true;
+        if (mbar_try_wait(a, parity)) return true;
         if (*ab.flag) return false;
         if (clock64() - t0 > limit_cycles) {
             *ab.flag = 1;
@@ -113,11 +94,10 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
 
 // Same, but never consults the abort flag: used only to drain work this
 // thread itself put in flight before the CTA exits.
-template <bool CLUSTER = false>
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) {
     const uint32_t a = smem_u32(bar);
     const long long t0 = clock64();
-    while (!(CLUSTER ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity))) {
+    while (!mbar_try_wait(a, parity)) {
         if (clock64() - t0 > kWaitLimitCycles) return false;
     }
     return true;
@@ -133,19 +113,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-
-// CTA-pair form of the same load: the data lands in this CTA's shared memory
-// and the completed bytes are counted on `bar_cluster`, a shared::cluster
-// address that may lie in the peer CTA of the pair (the pair's leader, whose
-// MMA reads both CTAs' halves). No multicast: each CTA loads its own half.
-__device__ __forceinline__ void tma_load_3d_pair(void *dst, const CUtensorMap *map,
-                                                 uint32_t bar_cluster, int c0, int c1, int c2) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile"
-        ".mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
 
@@ -205,103 +172,6 @@ __device__ __forceinline__ void tc_commit(uint64_t *bar) {
     asm volatile(
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             smem_u32(bar))
-        : "memory");
-}
-
-// ------------------------------------------------------------------ CTA pairs
-// Two CTAs of a cluster whose ranks differ in bit 0 form a pair: the leader
-// (even rank) issues MMAs of M = 256 whose A rows come half from each CTA's
-// shared memory (or tensor memory), whose B columns come half from each, and
-// whose accumulator rows land in each CTA's own tensor memory.
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-
-// shared::cluster address of this CTA's shared variable at `saddr` as seen in
-// the CTA of the cluster with rank `rank`.
-__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-
-// Arrive (release, cluster scope) on an mbarrier given by its shared::cluster
-// address, from lane 0 of the warp only.
-__device__ __forceinline__ void mbar_arrive_cluster_lane0(uint32_t bar_cluster, int lane) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.eq.s32 p, %1, 0;\n\t"
-        "@p mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n\t}" ::"r"(bar_cluster),
-        "r"(lane)
-        : "memory");
-}
-
-// Every thread of both CTAs of the cluster (a hardware barrier: both CTAs of
-// a cluster are resident together, so it always completes once both reach it).
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile(
-        "barrier.cluster.arrive.release.aligned;\n\t"
-        "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(dst_smem)),
-                 "r"(ncols)
-                 : "memory");
-}
-
-__device__ __forceinline__ void tmem_relinquish_pair() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
-                 : "memory");
-}
-
-// Arrive once on the barrier at the same shared-memory offset in both CTAs of
-// the pair when every pair MMA this thread issued so far has completed.
-__device__ __forceinline__ void tc_commit_pair_both(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-        " [%0], %1;" ::"r"(smem_u32(bar)),
-        "h"(static_cast<uint16_t>(3))
-        : "memory");
-}
-
-// The same, arriving on this CTA's barrier only.
-__device__ __forceinline__ void tc_commit_pair_local(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi,
-                                            uint32_t b_lo, uint32_t b_hi, uint32_t idesc,
-                                            uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-        "mov.b64 da, {%1, %2};\n\t"
-        "mov.b64 db, {%3, %4};\n\t"
-        "setp.ne.b32 p, %6, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], da, db, %5, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-__device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo,
-                                            uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 db;\n\t"
-        "mov.b64 db, {%2, %3};\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], db, %4, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -398,17 +268,22 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
     return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-// The two E4M3 codes of a 16-bit pair (low byte first) back to fp32, exactly.
-__device__ __forceinline__ uint64_t e4m3x2_to_f32x2(uint16_t v) {
-    uint32_t h;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(v));
-    float lo, hi;
-    asm("{.reg .f16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;}"
-        : "=f"(lo), "=f"(hi)
-        : "r"(h));
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
+// Adds the four E4M3 values of a packed quad (exactly: every E4M3 value is an
+// f16 value) to two fp32 sums, a the low and b the high value of each pair:
+// two conversions to f16 pairs and four mixed-precision f16 + f32 adds.
+__device__ __forceinline__ void acc_e4m3x4(uint32_t q4, float &a, float &b) {
+    uint32_t h01, h23;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"(static_cast<uint16_t>(q4)));
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"(static_cast<uint16_t>(q4 >> 16)));
+    asm("{.reg .f16 x0, x1, x2, x3;\n\t"
+        "mov.b32 {x0, x1}, %2;\n\t"
+        "mov.b32 {x2, x3}, %3;\n\t"
+        "add.rn.f32.f16 %0, x0, %0;\n\t"
+        "add.rn.f32.f16 %1, x1, %1;\n\t"
+        "add.rn.f32.f16 %0, x2, %0;\n\t"
+        "add.rn.f32.f16 %1, x3, %1;}"
+        : "+f"(a), "+f"(b)
+        : "r"(h01), "r"(h23));
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
