@@ -15,12 +15,15 @@
 //   n_eff  = #{t : T[t] <= last position / blk}          (later blocks unread)
 //   n_full = #{t : T[t] <= (first position + 1) / blk - 1} (no causal mask)
 //
-// Grid: one CTA per item, items ordered so that the CTAs resident together
-// cover a few tile pairs of every group and start the group's table at the
-// same time: they walk its blocks in lockstep, each block comes from HBM once
-// and then from L2. (A persistent stream-K schedule that balances the last
-// wave staggers the CTAs instead and read several times more DRAM; under the
-// 1 kW power cap that sustained runs reach, it was not faster either.) When
+// Grid: one CTA per item, items ordered group by group (all tile pairs of a
+// group, then the next group): the CTAs resident together hold every tile
+// pair of a few groups, start each group's table at the same time and walk
+// its blocks in lockstep, so each block comes from HBM once and then from L2,
+// and the items past the last full wave (split below) cover the last groups
+// whole, whose tables the full waves did not read. (A persistent stream-K
+// schedule that balances the last wave staggers the CTAs instead and read
+// several times more DRAM; under the 1 kW power cap that sustained runs
+// reach, it was not faster either.) When
 // the items do not fill the SMs evenly, the items past the last full wave are
 // cut into segments of their block lists (split-KV): each segment CTA writes a
 // normalised partial O and its LSE to the workspace and the item's last CTA
@@ -237,8 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int per_b = units * P.n_pairs;
     const int b = P.b_order[item / per_b];
     const int rem = item % per_b;
-    const int pair = rem / units;
-    const int unit = rem % units;
+    const int unit = rem / P.n_pairs;  // group by group
+    const int pair = rem % P.n_pairs;
     const int g = PERTILE ? unit / P.G : unit;     // KV head
     const int head0 = PERTILE ? unit : g * P.G;  // query head of packed row 0
     const int cs = P.chunk_start[b];
