@@ -984,6 +984,47 @@ def run_sweep(args, dev, stream, flush, graphed, timed_round_robin, agg, peak, g
     return out
 
 
+def run_attention_only(args, chunks):
+    """Table build + attention of the workload only, ``--warmup`` untimed and
+    ``--steps`` timed launches (L2 flushed before each): the command the
+    committed ncu summaries capture. Prints one JSON line with the
+    attention's median time; not a benchmark line."""
+    import torch
+
+    import serving_block_union_b200 as ca
+    import workloads
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    ca.load_library()
+    wl = chunks[-1]
+    if len(chunks) != 1:
+        raise SystemExit("--attention-only takes a single-chunk workload")
+    mask = workloads.make_mask(wl)
+    Q, K, V = (t.to(dev) for t in workloads.make_qkv(wl))
+    maskd = torch.from_numpy(mask).to(dev)
+    ws = ca.new_workspace(wl.B, wl.H_q, wl.H_kv, wl.C, wl.blk, device=dev)
+    T, c, _, _ = ca.build_block_tables(maskd, wl.group)
+    O = torch.empty_like(Q)
+    L = torch.empty((wl.B, wl.H_q, wl.C), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    times = []
+    for i in range(args.warmup + args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ca.build_block_tables(maskd, wl.group, tables=T, counts=c)
+        a.record()
+        ca.chunk_attention(Q, K, V, T, c, wl.chunk_start, O=O, LSE=L, workspace=ws)
+        b.record()
+        torch.cuda.synchronize(dev)
+        if i >= args.warmup:
+            times.append(a.elapsed_time(b))
+    assert ca.read_device_status(ws) == ca.CA_OK, "device status not OK"
+    print(json.dumps({"mode": "attention-only", "workload": wl.name,
+                      "attn_ms_median": statistics.median(times), "launches": len(times)}))
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -995,12 +1036,16 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the per-configuration sweep (the headline line only)")
+    ap.add_argument("--attention-only", action="store_true",
+                    help="run only the workload's table build + attention (for profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     chunks = step_chunks(args.workload)
     if args.impl == "reference":
         return run_reference(args, chunks[-1], args.workload)
+    if args.attention_only:
+        return run_attention_only(args, chunks)
     return run_ours(args, chunks)
 
 
