@@ -332,96 +332,6 @@ __global__ void __cluster_dims__(kClusterCtas, 1, 1) __launch_bounds__(kClusterT
     if (q == 0 && tid == 0) counts[bg] = n;
 }
 
-// One CTA per (b, g) with the same flat (row, unit) load order as the
-// cluster form, for many (b, g) (a batch of sequences): 256 threads, eight
-// 16-byte (or 32-bit) loads in flight per thread before they are folded into
-// shared memory with atomicOr, then one block-wide scan places the units'
-// entries. A (b, g) of 16 Q-blocks x 4 heads x 1040 KV blocks is 4160 loads,
-// about two DRAM round trips per thread; eight such CTAs fit an SM, so a
-// batch of 64 sequences at 128K (512 (b, g)) is one wave.
-constexpr int kFlatThreads = 256;
-constexpr int kFlatInFlight = 8;
-
-template <bool BITS>
-__global__ void __launch_bounds__(kFlatThreads)
-    union_tables_flat_kernel(const void *__restrict__ mask, int H_q, int nQ, int nKVmax, int G,
-                             int32_t *__restrict__ tables, int32_t *__restrict__ counts) {
-    __shared__ uint32_t s_bits[kMaxUnitsPerCta];
-    __shared__ int s_off[kMaxUnitsPerCta];
-    __shared__ int warp_sums[32];
-
-    constexpr int UB = BITS ? 32 : 16;  // KV blocks per unit
-    const int bg = blockIdx.x;
-    const int H_kv = H_q / G;
-    const int b = bg / H_kv, g = bg % H_kv;
-    const int tid = threadIdx.x;
-    const int nu = (nKVmax + UB - 1) / UB;
-    const int n_rows = G * nQ;
-    const size_t row0 = ((size_t)b * H_q + (size_t)g * G) * nQ;
-    int32_t *T = tables + (size_t)bg * nKVmax;
-
-    for (int u = tid; u < nu; u += kFlatThreads) s_bits[u] = 0;
-    __syncthreads();
-    const int pairs = n_rows * nu;
-    for (int p0 = tid; p0 < pairs; p0 += kFlatInFlight * kFlatThreads) {
-        uint32_t bits[kFlatInFlight];
-        int unit[kFlatInFlight];
-#pragma unroll
-        for (int k = 0; k < kFlatInFlight; ++k) {
-            const int p = p0 + k * kFlatThreads;
-            bits[k] = 0;
-            unit[k] = 0;
-            if (p < pairs) {
-                const int row = p / nu;
-                const int u = p - row * nu;
-                unit[k] = u;
-                if constexpr (BITS) {
-                    bits[k] = __ldg(static_cast<const uint32_t *>(mask) + (row0 + row) * nu + u);
-                } else {
-                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(
-                        static_cast<const uint8_t *>(mask) + (row0 + row) * (size_t)nKVmax +
-                        (size_t)u * 16));
-                    bits[k] = nonzero_bytes16(v);
-                }
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < kFlatInFlight; ++k)
-            if (bits[k]) atomicOr(&s_bits[unit[k]], bits[k]);
-    }
-    __syncthreads();
-    if constexpr (BITS) {
-        // bits at or past nKVmax name no block
-        if (tid == 0 && nu > 0) {
-            const int valid = nKVmax - (nu - 1) * 32;
-            if (valid < 32) s_bits[nu - 1] &= (1u << valid) - 1u;
-        }
-        __syncthreads();
-    }
-    int run = 0;
-    for (int r0 = 0; r0 < nu; r0 += kFlatThreads) {
-        const int u = r0 + tid;
-        const int c = u < nu ? __popc(s_bits[u]) : 0;
-        int tot = 0;
-        const int off = block_exclusive_scan(c, tid, kFlatThreads, warp_sums, &tot);
-        if (u < nu) s_off[u] = run + off;
-        run += tot;
-        __syncthreads();  // warp_sums is reused by the next round
-    }
-    for (int u = tid; u < nu; u += kFlatThreads) {
-        uint32_t m = s_bits[u];
-        int w = s_off[u];
-        const int j0 = u * UB;
-        while (m) {
-            const int k = __ffs(m) - 1;
-            T[w++] = j0 + k;
-            m &= m - 1;
-        }
-    }
-    for (int t = run + tid; t < nKVmax; t += kFlatThreads) T[t] = -1;
-    if (tid == 0) counts[bg] = run;
-}
-
 // Units per CTA of the cluster form, or 0 where it does not apply. It pays
 // only while one CTA per (b, g) leaves most SMs idle (a single sequence or a
 // few): measured at 128K (G = 4, 16 Q-blocks), 8 (b, g) build in 10.8 us
@@ -482,12 +392,6 @@ int launch_build_tables_bits(const uint32_t *mask, int B, int H_q, int nQ, int n
         if (cudaGetLastError() != cudaSuccess) return CA_ERR_CUDA;
         return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
     }
-    if (nW <= kMaxUnitsPerCta) {
-        union_tables_flat_kernel<true><<<B * H_kv, kFlatThreads, 0, stream>>>(
-            mask, H_q, nQ, nKVmax, group, tables, counts);
-        if (cudaGetLastError() != cudaSuccess) return CA_ERR_CUDA;
-        return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
-    }
     int wpr = ((nW + 31) / 32) * 32;
     if (wpr > kMaxThreads) wpr = kMaxThreads;
     int rg = 512 / wpr;
@@ -511,12 +415,6 @@ int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax,
         union_tables_cluster_kernel<false><<<dim3(kClusterCtas, B * H_kv), kClusterThreads, 0,
                                              stream>>>(mask, H_q, nQ, nKVmax, group, upc, tables,
                                                        counts);
-        if (cudaGetLastError() != cudaSuccess) return CA_ERR_CUDA;
-        return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
-    }
-    if (vec && n_chunks <= kMaxUnitsPerCta) {
-        union_tables_flat_kernel<false><<<B * H_kv, kFlatThreads, 0, stream>>>(
-            mask, H_q, nQ, nKVmax, group, tables, counts);
         if (cudaGetLastError() != cudaSuccess) return CA_ERR_CUDA;
         return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
     }
