@@ -331,3 +331,31 @@ def test_python_binding_rejects_bad_tensors(cuda_ok):
         ca.dense_chunk_attention(Q, K, K, [0], 64)
     with pytest.raises(ca.CAError):
         ca.dense_chunk_attention(Q.to(torch.bfloat16), K, K, [250], 64)  # cs + C > L_max
+
+
+# ------------------------------------------------------- running-max rescales
+
+@pytest.mark.parametrize("dense", [False, True])
+def test_large_logit_jumps_between_blocks(cuda_ok, dense):
+    """Logits that jump by tens of nats from block to block (up and down, a
+    later block's maximum far above everything before it), so the online
+    softmax has to raise its running maximum and rescale O in tensor memory
+    many times, including jumps larger than its lazy threshold: every query
+    has a unit component along one direction and each KV block's keys a
+    block-constant component a_j along it, so the row's logits in block j sit
+    near a_j / sqrt(D)."""
+    B, H_q, H_kv, D, blk, C, L_max, cs = 1, 8, 2, 128, 128, 256, 1280, (1024,)
+    nK = L_max // blk
+    g = torch.Generator().manual_seed(77)
+    Q = torch.randn(B, H_q, C, D, generator=g) * 0.3
+    Q[..., 0] = 1.0
+    K = torch.randn(B, H_kv, L_max, D, generator=g) * 0.3
+    V = torch.randn(B, H_kv, L_max, D, generator=g)
+    a = torch.tensor([0.0, 200.0, -300.0, 700.0, 100.0, 1000.0, -800.0, 500.0, 1100.0, 40.0])
+    K[..., 0] = a.repeat_interleave(blk)[None, None, :]
+    Q, K, V = Q.to(torch.bfloat16), K.to(torch.bfloat16), V.to(torch.bfloat16)
+    mask = np.ones((B, H_q, C // blk, nK), np.uint8)
+    T, c, _, _ = oracle.block_tables(mask, H_q // H_kv)
+    O, L = _run_gpu(Q, K, V, T, c, cs, dense=dense, blk=blk)
+    O_ref, L_ref = oracle.attention(Q, K, V, cs, blk, None if dense else T, None if dense else c)
+    compare(O, L, O_ref, L_ref)
