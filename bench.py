@@ -616,6 +616,15 @@ def run_ours(args, chunks):
     lead_run = graphed(lambda: attend_k(n - 1))
     compact_run, tile_run = graphed(compact_step), graphed(tile_step)
     fp8_run, fp8_dense_run = graphed(fp8_attend), graphed(fp8_dense)
+    # The attention kernel timed alone (its own loop, the same flush before
+    # every launch, before the long round robin below heats the GPU): the
+    # figure the burst peak of a kernel timed alone applies to. The
+    # round-robin figure, inside a long mixed step, is set against the
+    # sustained peak.
+    with ClockSampler(gpu_index) as clk_alone:
+        (alone_ms,) = timed_round_robin([attn_run], args.steps, args.warmup)
+    clocks_alone = clk_alone.summary()
+    assert ca.read_device_status(ws) == ca.CA_OK, "device status not OK"
     # Every path is timed in each step, round robin, so that all of them see
     # the same clocks and power state (a path timed alone in its own loop gets
     # whatever the loops before it left: the 1 kW power cap lowers the clocks
@@ -629,14 +638,7 @@ def run_ours(args, chunks):
              build_stress_bits], args.steps, args.warmup, lead=lead_run)
     clocks = clk.summary()
     assert ca.read_device_status(ws) == ca.CA_OK, "device status not OK"
-    # The attention kernel timed alone (its own loop, the same flush before
-    # every launch, after the round robin): the figure the burst peak of a
-    # kernel timed alone applies to. The round-robin figure, inside a long
-    # mixed step, is set against the sustained peak.
-    with ClockSampler(gpu_index) as clk_alone:
-        (alone_ms,) = timed_round_robin([attn_run], args.steps, args.warmup)
-    clocks_alone = clk_alone.summary()
-    assert ca.read_device_status(ws) == ca.CA_OK, "device status not OK"
+
 
     # End to end through the public API with pinned host buffers: per chunk its
     # mask, queries and new K/V rows go up, O and LSE come back. The copies run
@@ -837,7 +839,8 @@ def run_ours(args, chunks):
                      "unit": "TFLOP/s", "frac": alone_tflops / peak,
                      "traffic": profiled_traffic(name) if n == 1 else None,
                      "peak_source": f"{peak_kind} bf16 burst: the kernel timed alone in its "
-                                    f"own loop of {K_} launches, L2 flushed before each",
+                                    f"own loop of {K_} launches, L2 flushed before each, "
+                                    "before the round robin",
                      "ms_per_launch": total_alone / K_ / n,
                      "clocks": clocks_alone,
                      "in_step": {"achieved": attn_tflops, "peak": peak_sus,
