@@ -88,7 +88,12 @@ int check_attention(const void *Q, const void *K, const void *V, const int32_t *
 // split that makes those segment waves shortest. Each segment CTA writes a
 // normalised fp32 partial O and its base-2 LSE to the workspace; the last of
 // an item's CTAs to finish merges them (workspace counters, no waiting).
+// The kernel keeps a split item whole where its table prefix is shorter than
+// kMinSegEntries blocks per segment (measured on B200 at split 4: segments of
+// ~20 blocks cost 5-12% against the unsplit launch, ~33 break even, ~50 gain
+// 4%); the host cannot see the table lengths, the kernel can.
 constexpr int kMaxSplit = 8;
+constexpr int kMinSegEntries = 40;
 constexpr int kRowsPerItem = 256;     // packed rows of one item (two tiles)
 constexpr int kSplitMinBlocks = 64;   // items shorter than this are not split
 

@@ -263,38 +263,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int jlast = p_max / BLK;
     const int jfull = (p_min + 1) / BLK - 1;
 
-    if (threadIdx.x == 0) {
-        mbar_init(q_full, 1);
-        for (int s = 0; s < NST; ++s) {
-            mbar_init(k_full + s, 1);
-            mbar_init(k_empty + s, 1);
-            mbar_init(v_full + s, 1);
-            mbar_init(v_empty + s, 1);
-        }
-        for (int t = 0; t < 2; ++t) {
-            mbar_init(s_full + t, 1);
-            for (int c = 0; c < NPC; ++c) mbar_init(p_full + t * NPC + c, 4);
-            mbar_init(o_full + t, 1);
-        }
-        mbar_init(mma_done, 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == kTmaWarp && lane == 0) {
-        tma_prefetch_desc(&tmQ);
-        tma_prefetch_desc(&tmK);
-        tma_prefetch_desc(&tmV);
-    }
-    if (warp == kMmaWarp) {
-        tmem_alloc(tmem_slot, kTmemCols);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    const AbortState ab{abort_flag, P.status};
-
     // ---- table prefix this item walks (every role computes it the same way)
     const int32_t *T = nullptr;
     int base = 0;  // paged form: entries are base + block index
@@ -329,9 +297,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         n_eff = count_le<PERTILE>(T, cnt, jlast, lane, base);
         n_full = count_le<PERTILE>(T, n_eff, jfull, lane, base);
     }
+    // A split item whose prefix is short is not split after all: segments of
+    // fewer than kMinSegEntries blocks each cost more in their own prologue,
+    // epilogue and merge than they save (the table's length is known only
+    // here, on the device). Every segment of the item reads the same count, so
+    // all agree; segment 0 then takes the whole item and the others leave
+    // before they touch shared memory, TMEM or the merge counters.
+    if (nseg > 1 && n_eff < kMinSegEntries * nseg) {
+        if (seg > 0) return;
+        nseg = 1;
+    }
     // this CTA's segment of the prefix: table entries [t0, t0 + n_run)
     const int t0 = (int)((long long)seg * n_eff / nseg);
     const int n_run = (int)((long long)(seg + 1) * n_eff / nseg) - t0;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < NST; ++s) {
+            mbar_init(k_full + s, 1);
+            mbar_init(k_empty + s, 1);
+            mbar_init(v_full + s, 1);
+            mbar_init(v_empty + s, 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(s_full + t, 1);
+            for (int c = 0; c < NPC; ++c) mbar_init(p_full + t * NPC + c, 4);
+            mbar_init(o_full + t, 1);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == kTmaWarp && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+    }
+    if (warp == kMmaWarp) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const AbortState ab{abort_flag, P.status};
 
     // Role code sits inside the branch that re-sized its registers, so the
     // compiler allocates each role within its own budget.
@@ -749,7 +759,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             softmax_bar_sync();
             if (threadIdx.x == 0) {
                 const unsigned prev = atomicAdd(P.counters + rest, 1u);
-                *last_flag = prev + 1 == (unsigned)P.split;
+                *last_flag = prev + 1 == (unsigned)nseg;
             }
             softmax_bar_sync();
             if (*last_flag) {
@@ -758,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float mx = -INFINITY;
 #pragma unroll
                 for (int sg = 0; sg < kMaxSplit; ++sg) {
-                    ls[sg] = sg < P.split ? __ldcg(P.part_lse + row0 + (size_t)sg * kRowsPerItem)
+                    ls[sg] = sg < nseg ? __ldcg(P.part_lse + row0 + (size_t)sg * kRowsPerItem)
                                        : -INFINITY;
                     mx = fmaxf(mx, ls[sg]);
                 }
@@ -774,7 +784,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float acc[32];
 #pragma unroll
                     for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-                    for (int sg = 0; sg < P.split; ++sg) {
+                    for (int sg = 0; sg < nseg; ++sg) {
                         const float w = ls[sg] * inv_w;
                         const float4 *src = reinterpret_cast<const float4 *>(
                             P.part_o + (row0 + (size_t)sg * kRowsPerItem) * D + c * 32);

@@ -118,33 +118,67 @@ def test_tiny_workload_tables_from_gpu_builder(cuda_ok):
 # ------------------------------------------------------- split of the last wave
 
 SPLIT = [
-    # B, H_q, H_kv, D, blk, C, L_max, chunk_start: few items over long caches,
-    # so the launch cuts every item into segments merged through the workspace
-    (1, 4, 1, 128, 64, 256, 64 * 80, (64 * 76,)),        # 4 items -> 8 segments each
-    (2, 8, 2, 64, 128, 384, 128 * 72, (128 * 64, 128 * 64)),
-    (1, 32, 8, 128, 128, 128, 128 * 70, (128 * 69,)),    # G = 4, 16 items
+    # B, H_q, H_kv, D, blk, C, L_max, chunk_start, density: few items over
+    # long caches, so the launch cuts every item into segments merged through
+    # the workspace (each segment at least 40 table entries long)
+    (1, 4, 1, 128, 64, 256, 64 * 400, (64 * 396,), 0.3),      # 4 items -> 8 segments each
+    (2, 8, 2, 64, 128, 384, 128 * 300, (128 * 292, 128 * 292), 0.3),  # 24 items -> 6 each
+    (1, 32, 8, 128, 128, 128, 128 * 380, (128 * 379,), 0.6),  # G = 4, 16 items -> 8 each
 ]
 
+# entries a split item's segments must each walk, else the kernel keeps the
+# item whole (the library's kMinSegEntries)
+MIN_SEG_ENTRIES = 40
 
-@pytest.mark.parametrize("case", SPLIT)
-def test_split_last_wave_full_compare(cuda_ok, case):
-    B, H_q, H_kv, D, blk, C, L_max, cs = case
-    mask, Q, K, V = _small_case(B, H_q, H_kv, D, blk, C, L_max, cs, 0.3, seed=sum(case[:7]))
+
+def _split_layout(n_items, n_sms):
+    """(n_first, split, byte offset of the partial-LSE slots) of a launch: the
+    full waves stay whole, the split makes the remaining segment waves
+    shortest (the library's plan for one cache length)."""
+    n_first = (n_items // n_sms) * n_sms
+    n_rest = n_items - n_first
+    best, best_frac = 1, 1.0
+    for s in range(2, 9):
+        frac = -(-n_rest * s // n_sms) / s
+        if frac < best_frac:
+            best, best_frac = s, frac
+    return n_first, best, 256 + -(-4 * n_rest // 256) * 256
+
+
+def _run_split_case(B, H_q, H_kv, D, blk, C, L_max, cs, mask, Q, K, V):
+    """Runs the case on a full workspace whose partial-LSE slots start as NaN;
+    returns O, LSE, the tables, and for every split item (rest item order) the
+    segments that wrote their slots."""
     T, c, _, _ = oracle.block_tables(mask, H_q // H_kv)
     Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
     Td, cd = torch.from_numpy(T).cuda(), torch.from_numpy(c).cuda()
     ws = ca.new_workspace(B, H_q, H_kv, C, blk)
-    assert ws.numel() > 256  # room for the split on this device
+    G = H_q // H_kv
+    n_pairs = (-(-C // (128 // G)) + 1) // 2
+    items = B * H_kv * n_pairs
+    n_first, split, lse_off = _split_layout(items, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert n_first == 0 and split > 1  # every item is a split item
+    n_slot = items * split * 256
+    ws[lse_off:lse_off + 4 * n_slot] = 255  # NaN in every partial LSE slot
     O, L = ca.chunk_attention(Qd, Kd, Vd, Td, cd, cs, workspace=ws)
     assert ca.read_device_status(ws) == ca.CA_OK
     # every merge counter (one uint32 per split item, after the 256-byte
     # header) is back at zero, ready for the next call
-    G = H_q // H_kv
-    items = B * H_kv * ((-(-C // (128 // G)) + 1) // 2)
-    assert items < 148
     assert int(ws[256:256 + 4 * items].count_nonzero()) == 0
+    slots = ws[lse_off:lse_off + 4 * n_slot].view(torch.float32).view(items, split, 256)
+    wrote = ~torch.isnan(slots).all(dim=2)  # [item, segment]
+    return O, L, T, c, wrote.cpu().numpy(), ws, (Qd, Kd, Vd, Td, cd)
+
+
+@pytest.mark.parametrize("case", SPLIT)
+def test_split_last_wave_full_compare(cuda_ok, case):
+    B, H_q, H_kv, D, blk, C, L_max, cs, p = case
+    mask, Q, K, V = _small_case(B, H_q, H_kv, D, blk, C, L_max, cs, p, seed=sum(case[:7]))
+    O, L, T, c, wrote, ws, dev = _run_split_case(B, H_q, H_kv, D, blk, C, L_max, cs, mask, Q, K, V)
+    assert wrote.all()  # every segment of every item ran and wrote its partial
     O_ref, L_ref = oracle.attention(Q, K, V, cs, blk, T, c)
     compare(O, L, O_ref, L_ref)
+    Qd, Kd, Vd, Td, cd = dev
     # the same call on a minimal workspace runs unsplit: same result within rounding
     ws_min = torch.zeros(256, dtype=torch.uint8, device="cuda")
     O1, L1 = ca.chunk_attention(Qd, Kd, Vd, Td, cd, cs, workspace=ws_min)
@@ -155,8 +189,33 @@ def test_split_last_wave_full_compare(cuda_ok, case):
     assert torch.equal(O, O2) and torch.equal(L, L2)
 
 
+def test_split_only_long_items(cuda_ok):
+    """Groups 0-3 select most of a 380-block cache, groups 4-7 about a third:
+    the long groups' items run as 8 segments merged in the kernel, the short
+    ones (fewer than 40 entries per segment) stay whole on their first
+    segment's CTA while the other segments leave at once; all rows match the
+    oracle and no merge counter is left set."""
+    B, H_q, H_kv, D, blk, C, L_max, cs = 1, 32, 8, 128, 128, 128, 128 * 380, (128 * 379,)
+    mask, Q, K, V = _small_case(B, H_q, H_kv, D, blk, C, L_max, cs, 0.6, seed=77)
+    thin = np.random.default_rng(78).random(mask[:, 16:].shape) < 0.15
+    mask[:, 16:] &= thin.astype(np.uint8)  # heads 16-31 (groups 4-7): density 0.09
+    O, L, T, c, wrote, ws, _ = _run_split_case(B, H_q, H_kv, D, blk, C, L_max, cs, mask, Q, K, V)
+    split = wrote.shape[1]
+    n_pairs = wrote.shape[0] // H_kv
+    for item in range(wrote.shape[0]):
+        g = item // n_pairs  # one sequence: items run group by group
+        # every item walks its group's whole table (the cache ends at the chunk)
+        if c[0, g] >= MIN_SEG_ENTRIES * split:
+            assert wrote[item].all(), (item, int(c[0, g]))
+        else:
+            assert not wrote[item].any(), (item, int(c[0, g]))
+    assert c[0, :4].min() >= MIN_SEG_ENTRIES * split and c[0, 4:].max() < MIN_SEG_ENTRIES * split
+    O_ref, L_ref = oracle.attention(Q, K, V, cs, blk, T, c)
+    compare(O, L, O_ref, L_ref)
+
+
 def test_split_dense_full_compare(cuda_ok):
-    B, H_q, H_kv, D, blk, C, L_max, cs = SPLIT[0]
+    B, H_q, H_kv, D, blk, C, L_max, cs, _ = SPLIT[0]
     _, Q, K, V = _small_case(B, H_q, H_kv, D, blk, C, L_max, cs, 0.0, seed=31)
     O, L = _run_gpu(Q, K, V, None, None, cs, dense=True, blk=blk)
     O_ref, L_ref = oracle.attention(Q, K, V, cs, blk)

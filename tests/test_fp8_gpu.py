@@ -50,7 +50,7 @@ SMALL = [
     (2, 8, 2, 64, 320, 1280, (448, 64)),
     (1, 32, 8, 128, 512, 2048, (1536,)),
     (2, 8, 8, 128, 200, 768, (512, 128)),     # G = 1, ragged chunk
-    (1, 16, 2, 64, 128, 64 * 90, (64 * 80,)),  # G = 8, long cache: the last wave is split
+    (1, 16, 2, 64, 128, 64 * 400, (64 * 390,)),  # G = 8, long cache: the last wave is split
 ]
 
 

@@ -15,9 +15,10 @@ pytestmark = pytest.mark.gpu
 
 
 def test_captured_step_matches_eager_and_oracle(cuda_ok):
-    wl = workloads.Workload("graph", B=1, H_q=8, H_kv=2, D=128, blk=128, C=512,
-                            L_max=128 * 80, chunk_start=(128 * 76,), seed=12,
-                            mask_kind="stripes", n_stripes=8, noise=0.02)
+    # 8 items over a 400-block cache, tables ~99% full: every item is split
+    wl = workloads.Workload("graph", B=1, H_q=8, H_kv=2, D=128, blk=128, C=256,
+                            L_max=128 * 400, chunk_start=(128 * 396,), seed=12,
+                            mask_kind="bernoulli", density=0.5)
     mask = torch.from_numpy(workloads.make_mask(wl)).cuda()
     Q, K, V = (t.cuda() for t in workloads.make_qkv(wl))
     ws = ca.new_workspace(wl.B, wl.H_q, wl.H_kv, wl.C, wl.blk)

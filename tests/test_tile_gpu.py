@@ -68,8 +68,10 @@ def test_small_shapes_tables_and_attention(cuda_ok, case, p):
 def test_split_last_wave(cuda_ok):
     """Few per-head items over a long cache: segments merged through the
     workspace, checked against the oracle in full."""
-    B, H_q, H_kv, D, blk, C, L_max, cs = 1, 4, 2, 128, 128, 512, 128 * 80, (128 * 76,)
-    mask, Q, K, V = _small_case(B, H_q, H_kv, D, blk, C, L_max, 0.3, seed=41)
+    B, H_q, H_kv, D, blk, C, L_max, cs = 1, 4, 2, 128, 128, 512, 128 * 400, (128 * 396,)
+    # dense enough that every item's table (about 400 entries) makes
+    # segments of at least 40 entries
+    mask, Q, K, V = _small_case(B, H_q, H_kv, D, blk, C, L_max, 0.9, seed=41)
     ws = ca.new_workspace(B, H_q, H_kv, C, blk)
     _, _, O, L = _gpu_tile(mask, Q, K, V, cs, blk, ws=ws)
     assert ca.read_device_status(ws) == ca.CA_OK

@@ -93,9 +93,9 @@ def test_noalloc_status_set_by_bad_count_then_cleared(cuda_ok):
 
 
 def test_noalloc_runs_a_split_shape_unsplit(cuda_ok):
-    # one sequence, 80 KV blocks, 4 work items: the workspace path cuts each
-    # item into segments; the 4 KB scratch has no room for that
-    B, H_q, H_kv, D, blk, C, L_max, cs = 1, 4, 1, 128, 64, 256, 64 * 80, (64 * 76,)
+    # one sequence, 400 KV blocks, 4 work items: the workspace path cuts each
+    # item into 8 segments; the 4 KB scratch has no room for that
+    B, H_q, H_kv, D, blk, C, L_max, cs = 1, 4, 1, 128, 64, 256, 64 * 400, (64 * 396,)
     rng = np.random.default_rng(41)
     mask = (rng.random((B, H_q, C // blk, L_max // blk)) < 0.3).astype(np.uint8)
     g = torch.Generator().manual_seed(41)
