@@ -589,16 +589,7 @@ def run_ours(args, chunks):
     def merge():
         ca.merge_attention_states(m_parts, O=m_out[0], LSE=m_out[1])
 
-    # the table build at a size where bandwidth is measurable: 64 sequences of
-    # this shape at 128K (16 Q-blocks, 1040 KV blocks), 10% Bernoulli mask
-    st_B, st_nQ, st_nK = 64, 16, 1040
-    st_np = (np.random.default_rng(77).random((st_B, wl0.H_q, st_nQ, st_nK)) < 0.1).astype(
-        np.uint8)
-    st_mask = torch.from_numpy(st_np).to(dev)
-    st_bits = torch.from_numpy(workloads.pack_mask_bits(st_np).view(np.int32)).to(dev)
-    del st_np
-    st_T = torch.empty((st_B, wl0.H_kv, st_nK), dtype=torch.int32, device=dev)
-    st_c = torch.empty((st_B, wl0.H_kv), dtype=torch.int32, device=dev)
+    st_B, st_nQ, st_nK, st_mask, st_bits, st_T, st_c = build_stress_inputs(wl0, dev)
 
     def build_stress():
         ca.build_block_tables(st_mask, wl0.group, tables=st_T, counts=st_c)
@@ -995,6 +986,56 @@ def run_sweep(args, dev, stream, flush, graphed, timed_round_robin, agg, peak, g
     return out
 
 
+def build_stress_inputs(wl, dev):
+    """The table build at a size where bandwidth is measurable: 64 sequences
+    of ``wl``'s head shape at 128K (16 Q-blocks, 1040 KV blocks), a 10%
+    Bernoulli mask as bytes and bit-packed, and the output buffers."""
+    import torch
+
+    import workloads
+    B, nQ, nK = 64, 16, 1040
+    m = (np.random.default_rng(77).random((B, wl.H_q, nQ, nK)) < 0.1).astype(np.uint8)
+    mask = torch.from_numpy(m).to(dev)
+    bits = torch.from_numpy(workloads.pack_mask_bits(m).view(np.int32)).to(dev)
+    T = torch.empty((B, wl.H_kv, nK), dtype=torch.int32, device=dev)
+    c = torch.empty((B, wl.H_kv), dtype=torch.int32, device=dev)
+    return B, nQ, nK, mask, bits, T, c
+
+
+def run_build_stress_only(args, chunks):
+    """The bench's table-build stress point only (byte mask, then bit-packed),
+    ``--warmup`` untimed and ``--steps`` timed calls each, L2 flushed before
+    each: the command the committed ncu summary of the build captures.
+    Prints one JSON line with the median times; not a benchmark line."""
+    import torch
+
+    import serving_block_union_b200 as ca
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    ca.load_library()
+    wl = chunks[-1]
+    B, nQ, nK, mask, bits, T, c = build_stress_inputs(wl, dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    out = {}
+    for name, call in (("bytes", lambda: ca.build_block_tables(mask, wl.group, tables=T, counts=c)),
+                       ("bits", lambda: ca.build_block_tables_bits(bits, nK, wl.group, tables=T,
+                                                                   counts=c))):
+        times = []
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            call()
+            b.record()
+            torch.cuda.synchronize(dev)
+            if i >= args.warmup:
+                times.append(a.elapsed_time(b) * 1e3)
+        out[name + "_us_median"] = statistics.median(times)
+    print(json.dumps({"mode": "build-stress-only", "B": B, "nQ": nQ, "nKVmax": nK, **out}))
+    return 0
+
+
 def run_attention_only(args, chunks):
     """Table build + attention of the workload only, ``--warmup`` untimed and
     ``--steps`` timed launches (L2 flushed before each): the command the
@@ -1049,6 +1090,8 @@ def main(argv=None):
                     help="skip the per-configuration sweep (the headline line only)")
     ap.add_argument("--attention-only", action="store_true",
                     help="run only the workload's table build + attention (for profiling)")
+    ap.add_argument("--build-stress-only", action="store_true",
+                    help="run only the table-build stress point (for profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -1057,6 +1100,8 @@ def main(argv=None):
         return run_reference(args, chunks[-1], args.workload)
     if args.attention_only:
         return run_attention_only(args, chunks)
+    if args.build_stress_only:
+        return run_build_stress_only(args, chunks)
     return run_ours(args, chunks)
 
 

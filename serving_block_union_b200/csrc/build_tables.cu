@@ -6,20 +6,27 @@
 // per-(batch, KV-group) table T_{b,g}; the CSR form is the kv_indptr /
 // kv_indices metadata handed to the paged kernel.
 //
-// Two forms. With few (b, g), each is spread over a cluster of CTAs (the
-// cluster kernel below). Otherwise one CTA per (b, g): thread (rg, c) owns 16
-// consecutive KV blocks (chunk c)
-// and ORs 16-byte vectors of the mask rows rg, rg + RG, ... of the group's
-// G * nQ rows (coalesced: consecutive threads read consecutive 16-byte words
-// of a row). Row groups are OR-combined through shared memory, every chunk
-// turns its 16 bytes into a 16-bit set, and a block-wide exclusive prefix sum
-// of the popcounts (warp shuffles + one shared-memory pass) gives each chunk
-// its write offset, so the table comes out ascending without a sort.
+// Three forms. With few (b, g), each is spread over a cluster of CTAs (the
+// cluster kernel below). With many, one CTA per (b, g) reads the group's
+// contiguous G * nQ mask rows with bulk copies into shared memory (the bulk
+// kernel below). Where neither applies (rows not 16-byte multiples, or wider
+// than the bulk form takes), one CTA per (b, g) reads with register loads:
+// thread (rg, c) owns 16 consecutive KV blocks (chunk c) and ORs 16-byte
+// vectors of the mask rows rg, rg + RG, ... of the group's rows (coalesced:
+// consecutive threads read consecutive 16-byte words of a row). Row groups
+// are OR-combined through shared memory, every chunk turns its 16 bytes into
+// a 16-bit set, and a block-wide exclusive prefix sum of the popcounts (warp
+// shuffles + one shared-memory pass) gives each chunk its write offset, so
+// the table comes out ascending without a sort.
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <type_traits>
+
 #include "ca_internal.h"
+#include "sm100_ptx.cuh"
 
 namespace ca {
 
@@ -201,6 +208,151 @@ __global__ void __launch_bounds__(kMaxThreads)
     if (tid == 0) counts[bg] = n;
 }
 
+// Bulk-copy form of the one-CTA-per-(b, g) union, for many (b, g) (a batch
+// of sequences). A (b, g)'s G * nQ mask rows are contiguous in memory, so the
+// CTA reads them as pieces of `rpp` whole rows, one cp.async.bulk copy per
+// piece into a two-stage shared-memory ring (completion counted in bytes on
+// the stage's mbarrier): two pieces, up to 64 KB, in flight per CTA without a
+// register per byte, against a few loads per thread in the register form.
+// Thread t ORs units t, t + 256, ... (16-byte vectors of a byte mask, or
+// 32-bit words of a bit-packed one) over every row of every piece; a
+// block-wide scan of the units' popcounts, in unit order, places each
+// unit's entries (ascending without a sort). Every wait is bounded: a piece
+// that never lands (not seen in practice) leaves the CTA's count at -1,
+// which the attention kernels reject, after the copies it issued are drained.
+constexpr int kBulkThreads = 256;
+constexpr int kBulkPieceBytes = 32 * 1024;  // one stage of the ring
+constexpr int kBulkMaxUnitsPerThread = 4;   // units per row <= 1024
+
+__device__ __forceinline__ void or_into(uint4 &a, const uint4 &v) {
+    a.x |= v.x;
+    a.y |= v.y;
+    a.z |= v.z;
+    a.w |= v.w;
+}
+__device__ __forceinline__ void or_into(uint32_t &a, uint32_t v) { a |= v; }
+
+// Bounded wait on phase `parity` of `bar`; false once the CTA's abort flag is
+// set or this wait has run past kWaitLimitCycles (it then sets the flag).
+__device__ __forceinline__ bool bulk_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
+    const uint32_t a = smem_u32(bar);
+    if (mbar_try_wait(a, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait(a, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
+template <bool BITS, int UPT>
+__global__ void __launch_bounds__(kBulkThreads)
+    union_tables_bulk_kernel(const void *__restrict__ mask, int H_q, int nQ, int nKVmax, int G,
+                             int rpp, int32_t *__restrict__ tables,
+                             int32_t *__restrict__ counts) {
+    using Unit = typename std::conditional<BITS, uint32_t, uint4>::type;
+    constexpr int UB = BITS ? 32 : 16;  // KV blocks per unit
+    extern __shared__ uint8_t bulk_raw[];
+    __shared__ uint64_t full[2];
+    __shared__ int warp_sums[32];
+    __shared__ int s_abort;
+
+    const int bg = blockIdx.x, tid = threadIdx.x;
+    const int H_kv = H_q / G;
+    const int b = bg / H_kv, g = bg % H_kv;
+    const int n_rows = G * nQ;
+    const int n_units = (nKVmax + UB - 1) / UB;
+    const size_t row_bytes = (size_t)n_units * sizeof(Unit);
+    const uint8_t *src = static_cast<const uint8_t *>(mask) +
+                         ((size_t)b * H_q + (size_t)g * G) * nQ * row_bytes;
+    uint8_t *stage0 = bulk_raw + ((128u - (smem_u32(bulk_raw) & 127u)) & 127u);
+    const uint32_t stage_bytes = (uint32_t)((size_t)rpp * row_bytes);
+    const int n_pieces = (n_rows + rpp - 1) / rpp;
+    int32_t *T = tables + (size_t)bg * nKVmax;
+
+    if (tid == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        s_abort = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // thread 0 issues piece p (rows [p * rpp, ...)) into stage p & 1
+    int issued = 0;
+    auto issue = [&](int p) {
+        const int r0 = p * rpp;
+        const uint32_t bytes = (uint32_t)((size_t)min(rpp, n_rows - r0) * row_bytes);
+        uint64_t *bar = &full[p & 1];
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_load(stage0 + (p & 1) * stage_bytes, src + (size_t)r0 * row_bytes, bytes, bar);
+        issued = p + 1;
+    };
+    if (tid == 0) {
+        issue(0);
+        if (n_pieces > 1) issue(1);
+    }
+    Unit acc[UPT];
+#pragma unroll
+    for (int k = 0; k < UPT; ++k) acc[k] = Unit{};
+    int landed = 0;  // pieces this thread saw complete
+    for (int p = 0; p < n_pieces; ++p) {
+        // every thread reaches every barrier below, whether its wait held or not
+        if (bulk_wait(&full[p & 1], (p >> 1) & 1, &s_abort)) {
+            landed = p + 1;
+            const uint8_t *st = stage0 + (p & 1) * stage_bytes;
+            const int nr = min(rpp, n_rows - p * rpp);
+#pragma unroll 4
+            for (int r = 0; r < nr; ++r) {
+                const Unit *row = reinterpret_cast<const Unit *>(st + (size_t)r * row_bytes);
+#pragma unroll
+                for (int k = 0; k < UPT; ++k) {
+                    const int u = tid + k * kBulkThreads;
+                    if (u < n_units) or_into(acc[k], row[u]);
+                }
+            }
+        }
+        __syncthreads();  // stage p & 1 is free again
+        if (tid == 0 && p + 2 < n_pieces && !s_abort) issue(p + 2);
+    }
+    if (s_abort) {  // the barrier above made the flag visible to every thread
+        if (tid == 0) {
+            for (int p = landed; p < issued; ++p) mbar_wait_drain(&full[p & 1], (p >> 1) & 1);
+            counts[bg] = -1;
+        }
+        return;
+    }
+    int run = 0;
+#pragma unroll
+    for (int k = 0; k < UPT; ++k) {
+        const int u = tid + k * kBulkThreads;
+        uint32_t bits = 0;
+        if (u < n_units) {
+            if constexpr (BITS) {
+                bits = acc[k];
+                const int valid = nKVmax - u * 32;  // blocks this word can name
+                if (valid < 32) bits &= (1u << valid) - 1u;
+            } else {
+                bits = nonzero_bytes16(acc[k]);
+            }
+        }
+        int tot = 0;
+        const int off = block_exclusive_scan(__popc(bits), tid, kBulkThreads, warp_sums, &tot);
+        int w = run + off;
+        const int j0 = u * UB;
+        while (bits) {
+            T[w++] = j0 + __ffs(bits) - 1;
+            bits &= bits - 1;
+        }
+        run += tot;
+        __syncthreads();  // warp_sums is reused by the next round
+    }
+    for (int t = run + tid; t < nKVmax; t += kBulkThreads) T[t] = -1;
+    if (tid == 0) counts[bg] = run;
+}
+
 // Cluster form of the same union: a (b, g) row set is spread over a cluster of
 // kClusterCtas CTAs, CTA q taking units [q * upc, (q + 1) * upc) of the KV
 // range (a unit is 16 blocks of a byte mask, one 16-byte load per row, or 32
@@ -342,6 +494,59 @@ int cluster_upc(int n_units, int n_bg) {
     return upc <= kMaxUnitsPerCta ? upc : 0;
 }
 
+// Rows per piece of the bulk form, or 0 where it does not apply (a row wider
+// than a piece, more than four units per thread). Bit-packed rows are 4-byte
+// multiples, so there the pieces hold a multiple of four rows and start on
+// 16 bytes; the caller checks the region's own alignment. The piece count is
+// the least that fits, the rows spread evenly over it.
+int bulk_rpp(int n_rows, size_t row_bytes, int n_units, bool bits) {
+    if (n_units > kBulkThreads * kBulkMaxUnitsPerThread || row_bytes > (size_t)kBulkPieceBytes)
+        return 0;
+    int rpp = (int)(kBulkPieceBytes / row_bytes);
+    if (rpp >= n_rows) return n_rows;  // one piece
+    if (bits) rpp &= ~3;
+    if (rpp <= 0) return 0;
+    const int n_pieces = (n_rows + rpp - 1) / rpp;
+    int even = (n_rows + n_pieces - 1) / n_pieces;
+    if (bits) even = (even + 3) & ~3;  // still <= rpp, a multiple of 4
+    return even;
+}
+
+template <bool BITS, int UPT>
+int launch_bulk_t(const void *mask, int B, int H_q, int nQ, int nKVmax, int group, int rpp,
+                  size_t smem, int32_t *tables, int32_t *counts, cudaStream_t stream) {
+    auto kern = union_tables_bulk_kernel<BITS, UPT>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        2 * kBulkPieceBytes + 128);
+    });
+    if (attr_err != cudaSuccess) return CA_ERR_CUDA;
+    kern<<<B * (H_q / group), kBulkThreads, smem, stream>>>(mask, H_q, nQ, nKVmax, group, rpp,
+                                                            tables, counts);
+    return cudaGetLastError() == cudaSuccess ? CA_OK : CA_ERR_CUDA;
+}
+
+template <bool BITS>
+int launch_bulk(const void *mask, int B, int H_q, int nQ, int nKVmax, int group, int rpp,
+                int32_t *tables, int32_t *counts, cudaStream_t stream) {
+    const int n_rows = group * nQ;
+    const int n_units = BITS ? (nKVmax + 31) / 32 : nKVmax / 16;
+    const size_t row_bytes = (size_t)n_units * (BITS ? 4 : 16);
+    const int stages = rpp < n_rows ? 2 : 1;
+    const size_t smem = (size_t)stages * rpp * row_bytes + 128;
+    const int upt = (n_units + kBulkThreads - 1) / kBulkThreads;
+    if (upt <= 1)
+        return launch_bulk_t<BITS, 1>(mask, B, H_q, nQ, nKVmax, group, rpp, smem, tables,
+                                      counts, stream);
+    if (upt <= 2)
+        return launch_bulk_t<BITS, 2>(mask, B, H_q, nQ, nKVmax, group, rpp, smem, tables,
+                                      counts, stream);
+    return launch_bulk_t<BITS, 4>(mask, B, H_q, nQ, nKVmax, group, rpp, smem, tables, counts,
+                                  stream);
+}
+
 // CSR form: indptr[bg] = sum of counts before bg; indices = valid prefixes.
 __global__ void __launch_bounds__(256)
     csr_kernel(const int32_t *__restrict__ tables, const int32_t *__restrict__ counts, int n_bg,
@@ -392,6 +597,17 @@ int launch_build_tables_bits(const uint32_t *mask, int B, int H_q, int nQ, int n
         if (cudaGetLastError() != cudaSuccess) return CA_ERR_CUDA;
         return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
     }
+    // the bulk form where the (b, g) regions and pieces start on 16 bytes
+    const int n_rows = group * nQ;
+    if ((reinterpret_cast<uintptr_t>(mask) & 15u) == 0 && ((size_t)n_rows * nW) % 4 == 0) {
+        if (const int rpp = bulk_rpp(n_rows, (size_t)nW * 4, nW, true)) {
+            const int st = launch_bulk<true>(mask, B, H_q, nQ, nKVmax, group, rpp, tables,
+                                             counts, stream);
+            if (st != CA_OK) return st;
+            return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices,
+                              stream);
+        }
+    }
     int wpr = ((nW + 31) / 32) * 32;
     if (wpr > kMaxThreads) wpr = kMaxThreads;
     int rg = 512 / wpr;
@@ -416,6 +632,12 @@ int launch_build_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax,
                                              stream>>>(mask, H_q, nQ, nKVmax, group, upc, tables,
                                                        counts);
         if (cudaGetLastError() != cudaSuccess) return CA_ERR_CUDA;
+        return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
+    }
+    if (const int rpp = vec ? bulk_rpp(group * nQ, (size_t)nKVmax, n_chunks, false) : 0) {
+        const int st = launch_bulk<false>(mask, B, H_q, nQ, nKVmax, group, rpp, tables, counts,
+                                          stream);
+        if (st != CA_OK) return st;
         return launch_csr(tables, counts, B * H_kv, nKVmax, page_ids, indptr, indices, stream);
     }
     int chp = ((n_chunks + 31) / 32) * 32;

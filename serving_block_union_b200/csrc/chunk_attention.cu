@@ -31,7 +31,8 @@
 // merges them (an atomic counter, no waiting).
 //
 // FP8 (template flag): E4M3 Q, K, V, kind::f8f6f4 MMAs (K = 32 per step), P
-// rounded to E4M3 as 2^(x + 4) in TMEM (four values per column).
+// rounded to E4M3 as 2^(x + 4) in TMEM (four values per column); O and the
+// LSE are normalised by the fp32 sum of the unrounded P, as in the bf16 path.
 //
 // Warp roles (384 threads, one CTA per SM):
 //   warps 0-3  softmax + epilogue of tile 0 (thread = TMEM lane = packed row)
@@ -549,7 +550,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (PERTILE) tab_reg = lane < n_run ? __ldg(T + t0 + lane) : 0;
 
         float m_run = -INFINITY, l_run = 0.0f;
-        float lh_run = 0.0f;  // FP8: the same sum over the E4M3-rounded P
         bool ok = true;
         for (int j = 0; j < n_run; ++j) {
             int e_j = 0;
@@ -646,7 +646,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t sl2x2 = f2_pack(sl2, sl2);
             const uint64_t nm2 = f2_pack(kPBias - m_use, kPBias - m_use);
             uint64_t acc2[4];
-            float acch[2] = {0.0f, 0.0f};  // FP8: sums of the rounded P
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc2[k] = 0ull;
 #pragma unroll
@@ -662,14 +661,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t p2 = f2_pack(ex2_approx(f2_lo(x2)), ex2_approx(f2_hi(x2)));
                     acc2[i & 3] = f2_add(acc2[i & 3], p2);
                     if constexpr (F8) {
-                        // O is normalised by the sum of the E4M3 values P.V uses
-                        // (an exact convex combination of V rows); the LSE keeps
-                        // the fp32 sum
+                        // P.V takes P rounded to E4M3; O and the LSE are both
+                        // normalised by the fp32 sum of the unrounded P
                         if (i & 1) {
-                            const uint32_t q4 = pack_e4m3x4(f2_lo(p_prev), f2_hi(p_prev),
-                                                            f2_lo(p2), f2_hi(p2));
-                            pk[i >> 1] = q4;
-                            acc_e4m3x4(q4, acch[0], acch[1]);
+                            pk[i >> 1] = pack_e4m3x4(f2_lo(p_prev), f2_hi(p_prev), f2_lo(p2),
+                                                     f2_hi(p2));
                         } else {
                             p_prev = p2;
                         }
@@ -686,7 +682,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             acc2[0] = f2_add(f2_add(acc2[0], acc2[1]), f2_add(acc2[2], acc2[3]));
             l_run += f2_lo(acc2[0]) + f2_hi(acc2[0]);
-            if constexpr (F8) lh_run = lh_run * alpha + (acch[0] + acch[1]);
         }
         bool have_o = false;
         if (n_run > 0 && __all_sync(0xffffffffu, ok)) {
@@ -694,8 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             have_o = __all_sync(0xffffffffu, got);
             tc_fence_after();
         }
-        const float l_o = F8 ? lh_run : l_run;  // the sum O is normalised by
-        const float inv_l = l_o > 0.0f ? P.o_scale / l_o : 0.0f;
+        const float inv_l = l_run > 0.0f ? P.o_scale / l_run : 0.0f;
         const float lse2 = (l_run > 0.0f && have_o) ? m_run + log2f(l_run) - kPBias : -INFINITY;
         uint16_t *orow = P.O + (((size_t)b * P.H_q + h) * P.C + r) * D;
         float *lse_out = (valid && P.LSE != nullptr) ? P.LSE + ((size_t)b * P.H_q + h) * P.C + r

@@ -1,6 +1,6 @@
 // sm100_ptx.cuh — thin inline-PTX wrappers for the Blackwell (sm_100a) pieces
-// the kernels use: mbarriers with bounded waits, TMA tiled loads (no cluster
-// multicast anywhere), tcgen05 MMA / commit / TMEM alloc / TMEM load-store,
+// the kernels use: mbarriers with bounded waits, TMA tiled loads and untiled
+// bulk copies (no cluster multicast anywhere), tcgen05 MMA / commit / TMEM alloc / TMEM load-store,
 // and the shared-memory matrix descriptors of the 5th-generation tensor core.
 #pragma once
 
@@ -113,6 +113,18 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// Untiled bulk copy global -> shared of `bytes` bytes (both addresses 16-byte
+// aligned, `bytes` a multiple of 16), completion counted in bytes on `bar`.
+// No multicast.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
+                                          uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
 
@@ -266,24 +278,6 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
     return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
-}
-
-// Adds the four E4M3 values of a packed quad (exactly: every E4M3 value is an
-// f16 value) to two fp32 sums, a the low and b the high value of each pair:
-// two conversions to f16 pairs and four mixed-precision f16 + f32 adds.
-__device__ __forceinline__ void acc_e4m3x4(uint32_t q4, float &a, float &b) {
-    uint32_t h01, h23;
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h01) : "h"(static_cast<uint16_t>(q4)));
-    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h23) : "h"(static_cast<uint16_t>(q4 >> 16)));
-    asm("{.reg .f16 x0, x1, x2, x3;\n\t"
-        "mov.b32 {x0, x1}, %2;\n\t"
-        "mov.b32 {x2, x3}, %3;\n\t"
-        "add.rn.f32.f16 %0, x0, %0;\n\t"
-        "add.rn.f32.f16 %1, x1, %1;\n\t"
-        "add.rn.f32.f16 %0, x2, %0;\n\t"
-        "add.rn.f32.f16 %1, x3, %1;}"
-        : "+f"(a), "+f"(b)
-        : "r"(h01), "r"(h23));
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.

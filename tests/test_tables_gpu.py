@@ -39,10 +39,13 @@ def test_tables_bit_exact_on_workloads(cuda_ok, name):
     # B, H_q, nQ, nKVmax, G
     (1, 4, 4, 16, 4), (2, 8, 3, 37, 2), (3, 6, 5, 50, 3), (1, 8, 1, 9, 8),
     (2, 4, 2, 7, 1), (1, 32, 16, 16400, 4), (1, 2, 64, 3000, 2), (5, 16, 2, 1, 16),
-    # many (b, g): one CTA each instead of a cluster (the flat form; the last
-    # is a batch of 64 sequences at 128K); a KV range too long for the
-    # per-CTA shared memory of both
-    (24, 32, 4, 160, 4), (64, 32, 16, 1040, 4), (1, 2, 1, 131088, 2),
+    # many (b, g): one CTA each instead of a cluster, the bulk-copy form
+    # (one piece; three pieces, a batch of 64 sequences at 128K; 2, 3, 4 and
+    # 13 pieces through the two-stage ring, with 1, 2 and 4 units per thread);
+    # an odd width (the register form); a KV range too long for the bulk form
+    # and the cluster's shared memory
+    (24, 32, 4, 160, 4), (64, 32, 16, 1040, 4), (40, 8, 2, 8192, 8), (40, 4, 1, 16384, 4),
+    (45, 8, 5, 4096, 4), (40, 1, 37, 9600, 1), (40, 8, 3, 1000, 4), (1, 2, 1, 131088, 2),
 ])
 @pytest.mark.parametrize("p", [0.0, 0.01, 0.3, 1.0])
 def test_tables_random_shapes(cuda_ok, shape, p):
@@ -106,7 +109,11 @@ def test_bit_packed_mask_gives_the_same_tables(cuda_ok, name):
 
 @pytest.mark.parametrize("shape", [(1, 4, 3, 33, 1), (2, 8, 5, 64, 4), (1, 16, 2, 1, 8),
                                    (3, 6, 7, 100, 2), (20, 16, 2, 100, 4), (64, 32, 16, 1040, 4),
-                                   (1, 2, 1, 262200, 2)])
+                                   # bulk form over 4 and 2 pieces (rows a multiple
+                                   # of four per piece); rows * words not a multiple
+                                   # of four (the register form)
+                                   (40, 16, 16, 4096, 16), (40, 1, 37, 9600, 1),
+                                   (40, 8, 7, 96, 2), (1, 2, 1, 262200, 2)])
 def test_bit_packed_random_masks(cuda_ok, shape):
     B, H_q, nQ, nK, G = shape
     rng = np.random.default_rng(sum(shape))
