@@ -46,7 +46,7 @@ SWEEP = ["tiny", "llama8b_32k", "llama8b_128k_d2", "llama8b_128k_d5", "llama8b_1
          "llama8b_128k_d20", "batched", "full_prefill"]
 PROFILES = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = [os.path.join(ROOT, "serving_block_union_b200", "csrc", f)
-                  for f in ("chunk_attention.cu", "sm100_ptx.cuh")]
+                  for f in ("chunk_attention.cu", "sm100_ptx.cuh", "ca_internal.h")]
 
 
 def kernel_source_hash() -> str:
@@ -624,6 +624,12 @@ def run_ours(args, chunks):
         (alone_ms,) = timed_round_robin([attn_run], alone_steps, args.warmup)
     clocks_alone = clk_alone.summary()
     assert ca.read_device_status(ws) == ca.CA_OK, "device status not OK"
+    # bf16 and FP8 attention side by side in a short loop of their own (the
+    # same flush before each launch): the two kernels compared at the same
+    # clocks, outside the long round robin's power state
+    pair_bf16_ms, pair_fp8_ms = timed_round_robin([attn_run, fp8_run], alone_steps, args.warmup,
+                                                  lead=lead_run)
+    assert ca.read_device_status(ws) == ca.CA_OK, "device status not OK"
     # Every path is timed in each step, round robin, so that all of them see
     # the same clocks and power state (a path timed alone in its own loop gets
     # whatever the loops before it left: the 1 kW power cap lowers the clocks
@@ -822,7 +828,14 @@ def run_ours(args, chunks):
             "dense_ms": total_fp8_dense / K_,
             "speedup_vs_dense_fp8": total_fp8_dense / total_fp8,
             "speedup_vs_bf16_attention": total_attn / total_fp8,
-            "note": "Q, K, V per-tensor E4M3 (amax / 448 descale), same tables"},
+            "short_loop": {
+                "launches": len(pair_fp8_ms), "attn_ms": agg(pair_fp8_ms) / len(pair_fp8_ms),
+                "bf16_attn_ms": agg(pair_bf16_ms) / len(pair_bf16_ms),
+                "speedup_vs_bf16_attention": agg(pair_bf16_ms) / agg(pair_fp8_ms),
+                "note": "bf16 and FP8 alternating in a short loop of their own, before the "
+                        "round robin (the kernels at the same clocks, not power capped)"},
+            "note": "Q, K, V per-tensor E4M3 (amax / 448 descale), same tables; the top-level "
+                    "figures are from the round robin of every path"},
         "merge_states": _merge_line(m_out[0], total_merge / K_, big_out[0], total_merge_big / K_,
                                     peaks, peak_kind),
         "effective_tflop_per_step": flops / 1e12,
