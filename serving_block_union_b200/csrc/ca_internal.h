@@ -86,14 +86,15 @@ int check_attention(const void *Q, const void *K, const void *V, const int32_t *
 // The plan keeps the full waves [0, n_first) whole and cuts each remaining
 // item's block list into `split` segments run by separate CTAs, choosing the
 // split that makes those segment waves shortest. Each segment CTA writes a
-// normalised fp32 partial O and its base-2 LSE to the workspace; the last of
-// an item's CTAs to finish merges them (workspace counters, no waiting).
-// The kernel keeps a split item whole where its table prefix is shorter than
-// kMinSegEntries blocks per segment (measured on B200 at split 4: segments of
-// ~20 blocks cost 5-12% against the unsplit launch, ~33 break even, ~50 gain
-// 4%); the host cannot see the table lengths, the kernel can.
+// normalised partial O (bf16) and its base-2 LSE (fp32) to the workspace;
+// the last of an item's CTAs to finish merges them in fp32 (workspace
+// counters, no waiting). The kernel keeps a split item whole where its table
+// prefix is shorter than kMinSegEntries blocks per segment: measured on B200
+// at split 4, segments of ~22 blocks (2% density, full-prefill chunk 25)
+// gain nothing, ~33 (chunk 40) gain 2%, ~50 (5% density) 3%; the host
+// cannot see the table lengths, the kernel can.
 constexpr int kMaxSplit = 8;
-constexpr int kMinSegEntries = 40;
+constexpr int kMinSegEntries = 24;
 constexpr int kRowsPerItem = 256;     // packed rows of one item (two tiles)
 constexpr int kSplitMinBlocks = 64;   // items shorter than this are not split
 
@@ -128,7 +129,7 @@ inline SplitPlan plan_split(int n_items, int num_sms, int D, bool allow) {
     p.split = best_s;
     p.lse_off = kWorkspaceHeader + align256(4 * (size_t)n_rest);
     p.o_off = p.lse_off + align256(4 * rows);
-    p.bytes = p.o_off + 4 * rows * (size_t)D;
+    p.bytes = p.o_off + 2 * rows * (size_t)D;  // bf16 partial O
     return p;
 }
 

@@ -27,8 +27,8 @@
 // reach, it was not faster either.) When
 // the items do not fill the SMs evenly, the items past the last full wave are
 // cut into segments of their block lists (split-KV): each segment CTA writes a
-// normalised partial O and its LSE to the workspace and the item's last CTA
-// merges them (an atomic counter, no waiting).
+// normalised partial O (bf16) and its LSE (fp32) to the workspace and the
+// item's last CTA merges them in fp32 (an atomic counter, no waiting).
 //
 // FP8 (template flag): E4M3 Q, K, V, kind::f8f6f4 MMAs (K = 32 per step), P
 // rounded to E4M3 as 2^(x + 4) in TMEM (four values per column); O and the
@@ -100,7 +100,7 @@ struct Params {
     int n_items, n_first, split;  // split of the last wave (split == 1: none)
     unsigned int *counters;       // [n_items - n_first] finished segments per item
     float *part_lse;              // [n_rest][split][256] base-2 LSE of a segment's rows
-    float *part_o;                // [n_rest][split][256][D] normalised partial O
+    uint16_t *part_o;             // [n_rest][split][256][D] normalised partial O (bf16)
     float scale_log2;
     float o_scale;              // factor on O (the V descale of FP8 inputs, else 1)
     const int32_t *tables;      // or, in the paged form, kv_indices (global pages)
@@ -718,8 +718,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (lse_out) *lse_out = lse2 * kLn2;
         } else {
-            // Segment of a split item: its normalised O (fp32) and base-2 LSE
-            // go to the workspace, one slot row per packed row.
+            // Segment of a split item: its normalised O (bf16) and base-2 LSE
+            // (fp32) go to the workspace, one slot row per packed row.
             // (recomputed from the block index: nothing of the item decode has
             // to stay live across the block loop for this rare path)
             const int kseg = (int)blockIdx.x - P.n_first;
@@ -729,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int m_ = (warp & 3) * 32 + lane;
             const size_t row0 = (size_t)rest * P.split * kRowsPerItem + (warp / 4) * 128 + m_;
             const size_t mine = row0 + (size_t)seg_ * kRowsPerItem;
-            float *po = P.part_o + mine * D;
+            uint16_t *po = P.part_o + mine * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t v[32];
@@ -739,13 +739,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = 0u;
                 }
-                float4 *dst = reinterpret_cast<float4 *>(po + c * 32);
+                uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    dst[i] = make_float4(__uint_as_float(v[4 * i]) * inv_l,
-                                         __uint_as_float(v[4 * i + 1]) * inv_l,
-                                         __uint_as_float(v[4 * i + 2]) * inv_l,
-                                         __uint_as_float(v[4 * i + 3]) * inv_l);
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]) * inv_l,
+                                        __uint_as_float(v[2 * i + 1]) * inv_l);
+                uint4 *dst = reinterpret_cast<uint4 *>(po + c * 32);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
             }
             P.part_lse[mine] = lse2;
             // publish, count this segment in, and let the item's last CTA merge
@@ -780,15 +782,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
                     for (int sg = 0; sg < nseg; ++sg) {
                         const float w = ls[sg] * inv_w;
-                        const float4 *src = reinterpret_cast<const float4 *>(
+                        // eight bf16 per 16-byte load; a bf16 widens to fp32
+                        // by moving its bits to the high half
+                        const uint4 *src = reinterpret_cast<const uint4 *>(
                             P.part_o + (row0 + (size_t)sg * kRowsPerItem) * D + c * 32);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float4 x = __ldcg(src + i);
-                            acc[4 * i] = fmaf(w, x.x, acc[4 * i]);
-                            acc[4 * i + 1] = fmaf(w, x.y, acc[4 * i + 1]);
-                            acc[4 * i + 2] = fmaf(w, x.z, acc[4 * i + 2]);
-                            acc[4 * i + 3] = fmaf(w, x.w, acc[4 * i + 3]);
+                        for (int i = 0; i < 4; ++i) {
+                            const uint4 x = __ldcg(src + i);
+                            const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                acc[8 * i + 2 * k] =
+                                    fmaf(w, __uint_as_float(xw[k] << 16), acc[8 * i + 2 * k]);
+                                acc[8 * i + 2 * k + 1] = fmaf(
+                                    w, __uint_as_float(xw[k] & 0xffff0000u), acc[8 * i + 2 * k + 1]);
+                            }
                         }
                     }
                     if (valid) {
@@ -945,7 +953,7 @@ int launch_t(const AttnArgs &a, cudaStream_t stream) {
     P.split = plan.split;
     P.counters = reinterpret_cast<unsigned int *>(ws + kWorkspaceHeader);
     P.part_lse = reinterpret_cast<float *>(ws + plan.lse_off);
-    P.part_o = reinterpret_cast<float *>(ws + plan.o_off);
+    P.part_o = reinterpret_cast<uint16_t *>(ws + plan.o_off);
     const unsigned grid = static_cast<unsigned>(plan.n_first +
                                                 (n_items - plan.n_first) * plan.split);
     kern<<<grid, kThreads, L::kDynamic, stream>>>(tq, tk, tv, P);

@@ -120,7 +120,7 @@ def test_tiny_workload_tables_from_gpu_builder(cuda_ok):
 SPLIT = [
     # B, H_q, H_kv, D, blk, C, L_max, chunk_start, density: few items over
     # long caches, so the launch cuts every item into segments merged through
-    # the workspace (each segment at least 40 table entries long)
+    # the workspace (each segment at least 24 table entries long)
     (1, 4, 1, 128, 64, 256, 64 * 400, (64 * 396,), 0.3),      # 4 items -> 8 segments each
     (2, 8, 2, 64, 128, 384, 128 * 300, (128 * 292, 128 * 292), 0.3),  # 24 items -> 6 each
     (1, 32, 8, 128, 128, 128, 128 * 380, (128 * 379,), 0.6),  # G = 4, 16 items -> 8 each
@@ -128,7 +128,7 @@ SPLIT = [
 
 # entries a split item's segments must each walk, else the kernel keeps the
 # item whole (the library's kMinSegEntries)
-MIN_SEG_ENTRIES = 40
+MIN_SEG_ENTRIES = 24
 
 
 def _split_layout(n_items, n_sms):
@@ -192,7 +192,7 @@ def test_split_last_wave_full_compare(cuda_ok, case):
 def test_split_only_long_items(cuda_ok):
     """Groups 0-3 select most of a 380-block cache, groups 4-7 about a third:
     the long groups' items run as 8 segments merged in the kernel, the short
-    ones (fewer than 40 entries per segment) stay whole on their first
+    ones (fewer than 24 entries per segment) stay whole on their first
     segment's CTA while the other segments leave at once; all rows match the
     oracle and no merge counter is left set."""
     B, H_q, H_kv, D, blk, C, L_max, cs = 1, 32, 8, 128, 128, 128, 128 * 380, (128 * 379,)

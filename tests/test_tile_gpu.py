@@ -70,7 +70,7 @@ def test_split_last_wave(cuda_ok):
     workspace, checked against the oracle in full."""
     B, H_q, H_kv, D, blk, C, L_max, cs = 1, 4, 2, 128, 128, 512, 128 * 400, (128 * 396,)
     # dense enough that every item's table (about 400 entries) makes
-    # segments of at least 40 entries
+    # segments of at least 24 entries
     mask, Q, K, V = _small_case(B, H_q, H_kv, D, blk, C, L_max, 0.9, seed=41)
     ws = ca.new_workspace(B, H_q, H_kv, C, blk)
     _, _, O, L = _gpu_tile(mask, Q, K, V, cs, blk, ws=ws)
