@@ -70,7 +70,10 @@ int ca_version(void);
  *         (indices needs indptr). Bit-exact, deterministic.
  * Errors: CA_ERR_INVALID_ARG (NULL / non-positive), CA_ERR_SHAPE (group does
  * not divide H_q), CA_ERR_ALIGN (tables/counts/indptr/indices not 4-byte
- * aligned), CA_ERR_CUDA (launch failure).
+ * aligned), CA_ERR_CUDA (launch failure). On the device, with many (b, g),
+ * a (b, g) whose mask rows do not land in shared memory within the bounded
+ * wait (never seen in practice) gets count -1 and its table is left as it
+ * was; the attention calls reject such a count (status bit 0).
  */
 int ca_build_block_tables(const uint8_t *mask, int B, int H_q, int nQ, int nKVmax, int group,
                           int32_t *tables, int32_t *counts, int32_t *indptr, int32_t *indices,

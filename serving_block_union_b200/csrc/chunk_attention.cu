@@ -28,7 +28,9 @@
 // the items do not fill the SMs evenly, the items past the last full wave are
 // cut into segments of their block lists (split-KV): each segment CTA writes a
 // normalised partial O (bf16) and its LSE (fp32) to the workspace and the
-// item's last CTA merges them in fp32 (an atomic counter, no waiting).
+// item's last CTA merges them in fp32 (an atomic counter, no waiting). An
+// item whose table would give segments shorter than kMinSegEntries blocks
+// runs whole on its first segment's CTA (decided here, from the count).
 //
 // FP8 (template flag): E4M3 Q, K, V, kind::f8f6f4 MMAs (K = 32 per step), P
 // rounded to E4M3 as 2^(x + 4) in TMEM (four values per column); O and the
