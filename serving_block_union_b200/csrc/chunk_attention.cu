@@ -660,7 +660,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < CK / 2; ++i) {
                     const int e0 = c * CK + 2 * i;
                     const uint64_t x2 = f2_fma(f2_pack(s[e0], s[e0 + 1]), sl2x2, nm2);
-                    const uint64_t p2 = f2_pack(ex2_approx(f2_lo(x2)), ex2_approx(f2_hi(x2)));
+                    // FP8: every 4th pair on the FMA pipe (the FP8 products are
+                    // short, so the exponentials set the softmax: 2.3% faster
+                    // at 128K; in bf16 the same split was 4.8% slower)
+                    const uint64_t p2 =
+                        (F8 && (c * CK / 2 + i) % 4 == 3)
+                            ? exp2_poly2(x2)
+                            : f2_pack(ex2_approx(f2_lo(x2)), ex2_approx(f2_hi(x2)));
                     acc2[i & 3] = f2_add(acc2[i & 3], p2);
                     if constexpr (F8) {
                         // P.V takes P rounded to E4M3; O and the LSE are both

@@ -440,6 +440,28 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     return r;
 }
 
+// 2^x for a pair on the FMA and integer pipes instead of the MUFU unit.
+// Cody-Waite range reduction: adding 1.5 * 2^23 rounds x to the nearest
+// integer r (held in the low mantissa bits of t), f = x - r lies in
+// [-1/2, 1/2]; 2^f is a degree-3 polynomial (a minimax fit made for this
+// kernel, relative error at most 1.02e-4 over the interval), and 2^r is added
+// to its exponent field as an integer (the bits of t shifted up 23 places).
+// x is clamped at -127, where the result is +0; the softmax never passes
+// more than 8.5.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+    const uint64_t xc = f2_pack(fmaxf(f2_lo(x2), -127.0f), fmaxf(f2_hi(x2), -127.0f));
+    const uint64_t t = f2_add(xc, f2_pack(12582912.0f, 12582912.0f));
+    const uint64_t r = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
+    const uint64_t f = f2_fma(r, f2_pack(-1.0f, -1.0f), xc);
+    uint64_t p = f2_fma(f2_pack(0.055009059607982635f, 0.055009059607982635f), f,
+                        f2_pack(0.2422109693288803f, 0.2422109693288803f));
+    p = f2_fma(p, f, f2_pack(0.6932829022407532f, 0.6932829022407532f));
+    p = f2_fma(p, f, f2_pack(1.0f, 1.0f));
+    const uint32_t lo = __float_as_uint(f2_lo(t)) * 8388608u + __float_as_uint(f2_lo(p));
+    const uint32_t hi = __float_as_uint(f2_hi(t)) * 8388608u + __float_as_uint(f2_hi(p));
+    return f2_pack(__uint_as_float(lo), __uint_as_float(hi));
+}
+
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;

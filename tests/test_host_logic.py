@@ -114,3 +114,44 @@ def test_profiled_traffic_needs_matching_kernel_hash(tmp_path, monkeypatch):
     assert bench.kernel_source_hash() == h1
     src.write_text("int a; int c;\n")
     assert bench.kernel_source_hash() != h1
+
+
+def _poly_constants():
+    """The FMA-pipe exponential's coefficients, read from the kernel header
+    (so the test checks the constants the kernel compiles)."""
+    import re
+    src = open(os.path.join(os.path.dirname(__file__), "..", "serving_block_union_b200", "csrc",
+                            "sm100_ptx.cuh")).read()
+    body = src[src.index("exp2_poly2(uint64_t x2)"):]
+    body = body[:body.index("\n}\n")]
+    vals = [float(v) for v in re.findall(r"f2_pack\(([0-9.]+)f, \1f\)", body)]
+    # 1.5 * 2^23 (round shift), then c3, c2, c1, 1 in Horner order
+    return vals
+
+
+def test_fma_pipe_exp2_meets_its_stated_bound():
+    """exp2_poly2 (FP8 softmax, every 4th pair): the same float32 steps as
+    the device code; relative error at most 1.02e-4 against 2^x over the
+    softmax's range, +0 at the -127 clamp, positive and finite above it."""
+    vals = _poly_constants()
+    assert vals[0] == 12582912.0
+    c3, c2, c1, one = (np.float32(v) for v in vals[1:5])
+    assert one == 1.0
+    f32 = np.float32
+    x = np.concatenate([np.linspace(-127, 8.5, 2_000_001), [-127.0, -126.5, -0.5, 0.5, 8.5]])
+    x = np.maximum(x.astype(f32), f32(-127))
+    t = (x + f32(12582912.0)).astype(f32)
+    r = (t - f32(12582912.0)).astype(f32)
+    f = (x - r).astype(f32)
+
+    def fma(a, b, c):  # one rounding, as the device's fused multiply-add
+        return (a.astype(np.float64) * np.float64(b) + np.float64(c)).astype(f32)
+
+    p = fma(fma(fma(np.full_like(f, c3), f, c2), f, c1), f, one)
+    bits = (t.view(np.uint32).astype(np.uint64) * 8388608 + p.view(np.uint32)) % (1 << 32)
+    y = bits.astype(np.uint32).view(np.float32).astype(np.float64)
+    assert y[x == -127].max() == 0.0
+    ok = x > -126  # normal results
+    rel = np.abs(y[ok] / np.exp2(x[ok].astype(np.float64)) - 1)
+    assert rel.max() <= 1.02e-4
+    assert np.all(np.isfinite(y)) and np.all(y >= 0)
