@@ -232,22 +232,6 @@ __device__ __forceinline__ void or_into(uint4 &a, const uint4 &v) {
 }
 __device__ __forceinline__ void or_into(uint32_t &a, uint32_t v) { a |= v; }
 
-// Bounded wait on phase `parity` of `bar`; false once the CTA's abort flag is
-// set or this wait has run past kWaitLimitCycles (it then sets the flag).
-__device__ __forceinline__ bool bulk_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
-    const uint32_t a = smem_u32(bar);
-    if (mbar_try_wait(a, parity)) return true;
-    const long long t0 = clock64();
-    while (true) {
-        if (mbar_try_wait(a, parity)) return true;
-        if (*abort) return false;
-        if (clock64() - t0 > kWaitLimitCycles) {
-            *abort = 1;
-            return false;
-        }
-    }
-}
-
 template <bool BITS, int UPT>
 __global__ void __launch_bounds__(kBulkThreads)
     union_tables_bulk_kernel(const void *__restrict__ mask, int H_q, int nQ, int nKVmax, int G,
@@ -272,6 +256,7 @@ __global__ void __launch_bounds__(kBulkThreads)
     const uint32_t stage_bytes = (uint32_t)((size_t)rpp * row_bytes);
     const int n_pieces = (n_rows + rpp - 1) / rpp;
     int32_t *T = tables + (size_t)bg * nKVmax;
+    const AbortState ab{&s_abort, nullptr};  // a timeout shows as count -1
 
     if (tid == 0) {
         mbar_init(&full[0], 1);
@@ -300,7 +285,7 @@ __global__ void __launch_bounds__(kBulkThreads)
     int landed = 0;  // pieces this thread saw complete
     for (int p = 0; p < n_pieces; ++p) {
         // every thread reaches every barrier below, whether its wait held or not
-        if (bulk_wait(&full[p & 1], (p >> 1) & 1, &s_abort)) {
+        if (mbar_wait(&full[p & 1], (p >> 1) & 1, ab)) {
             landed = p + 1;
             const uint8_t *st = stage0 + (p & 1) * stage_bytes;
             const int nr = min(rpp, n_rows - p * rpp);

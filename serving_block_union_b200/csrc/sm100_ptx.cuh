@@ -70,12 +70,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // which every other wait of the CTA returns false at once.
 struct AbortState {
     volatile int *flag;        // shared memory
-    unsigned int *status;      // global workspace status word
+    unsigned int *status;      // global workspace status word, or null
 };
 
 // Waits until the phase with the given parity of `bar` has completed.
-// Returns false (and records kDevErrTimeout) if the wait exceeded the limit or
-// the CTA is aborting.
+// Returns false (and records kDevErrTimeout in the status word, if there is
+// one) if the wait exceeded the limit or the CTA is aborting.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const AbortState &ab,
                                           long long limit_cycles = kWaitLimitCycles) {
     const uint32_t a = smem_u32(bar);
@@ -86,7 +86,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const 
         if (*ab.flag) return false;
         if (clock64() - t0 > limit_cycles) {
             *ab.flag = 1;
-            atomicOr(ab.status, kDevErrTimeout);
+            if (ab.status != nullptr) atomicOr(ab.status, kDevErrTimeout);
             return false;
         }
     }
