@@ -309,6 +309,12 @@ __global__ void __launch_bounds__(kBulkThreads)
         }
         return;
     }
+    // The table is assembled in the ring's shared memory (free now: every
+    // piece has been consumed) where it fits, then written out with
+    // consecutive threads on consecutive entries; a unit's entries written
+    // straight to global memory would be one scattered 4-byte store each.
+    const bool in_smem = (size_t)nKVmax * 4 <= (n_pieces > 1 ? 2u : 1u) * (size_t)stage_bytes;
+    int32_t *dst = in_smem ? reinterpret_cast<int32_t *>(stage0) : T;
     int run = 0;
 #pragma unroll
     for (int k = 0; k < UPT; ++k) {
@@ -328,13 +334,17 @@ __global__ void __launch_bounds__(kBulkThreads)
         int w = run + off;
         const int j0 = u * UB;
         while (bits) {
-            T[w++] = j0 + __ffs(bits) - 1;
+            dst[w++] = j0 + __ffs(bits) - 1;
             bits &= bits - 1;
         }
         run += tot;
-        __syncthreads();  // warp_sums is reused by the next round
+        __syncthreads();  // warp_sums is reused by the next round; dst complete
     }
-    for (int t = run + tid; t < nKVmax; t += kBulkThreads) T[t] = -1;
+    if (in_smem) {
+        for (int t = tid; t < nKVmax; t += kBulkThreads) T[t] = t < run ? dst[t] : -1;
+    } else {
+        for (int t = run + tid; t < nKVmax; t += kBulkThreads) T[t] = -1;
+    }
     if (tid == 0) counts[bg] = run;
 }
 
