@@ -52,6 +52,12 @@ def test_workspace_bytes(lib):
     n = lib.ca_workspace_bytes(1, 32, 8, 2048, 128)
     assert n >= 16 and n % 256 == 0
     assert lib.ca_workspace_bytes(0, 32, 8, 2048, 128) == 0
+    # 128K headline shape on 148 SMs (the count used where no device can be
+    # read, and B200's): 256 work items, 148 whole, 108 cut into 4 segments;
+    # 256-byte header, one uint32 counter per split item (padded to 256 B),
+    # fp32 partial LSE and bf16 partial O per segment row (256 rows, D = 128)
+    rows = 108 * 4 * 256
+    assert n == 256 + 512 + 4 * rows + 2 * rows * 128
 
 
 # Fake device addresses: never dereferenced because every call below fails
